@@ -1,0 +1,333 @@
+#!/usr/bin/env python
+"""Benchmark of the SchNet energy/force hot path on B200.
+
+One step = one NVE velocity-Verlet step of 64 replicas of a 269-bead chain (r_cut 12 A,
+F 128, K 50 Gaussians, T 3 blocks): kick + drift, neighbour-list rebuild, energy and
+forces, kick.  That is every row of the hot path: neighbour build, radial basis, filter
+network, message passing + segmented sums, update/readout, the hand-derived backward, and
+the integrator.  The metric is energy+force evaluations per second (one per step) and
+directed edges per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Inputs are seeded synthetic chains (self-avoiding random walks, 3.8 A bonds, 20 bead
+types) and random weights from N(0, 1/fan_in), resident in HBM before timing.  L2 (126 MB)
+is flushed between timed steps by writing a 256 MiB buffer; each step is bracketed by CUDA
+events on the library's stream; the per-rank sum is max-reduced over ranks.  For N > 1 each
+rank runs its own batch of replicas (no collective on the data path; weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+import numpy as np  # noqa: E402
+
+from schnet_gnn_molecular_cell_b200 import synth  # noqa: E402
+
+METRIC = "energy+force evals/s and edges/s (1 B200); % of HBM/tensor roofline"
+CFG = 2
+MASS, DT, TEMP = 12.0, 2.0, 300.0
+WORKLOAD = "64 x 269-bead SAW chains, r_cut 12 A, SchNet F128 K50 T3: one velocity-Verlet step " \
+           "(neighbour rebuild + energy/forces + integration)"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_md_rate(w, v0, n_rep_sample: int, budget_s: float, min_steps: int = 1):
+    """Time the CPU oracle's velocity-Verlet steps on the first n_rep_sample replicas of the
+    workload; returns (evals/s scaled to the full workload, steps run, seconds, threads)."""
+    from oracle import oracle
+    n_per = w.system.n_per_replica
+    s = synth.SystemCfg(n_per, n_rep_sample, w.system.box)
+    n = n_per * n_rep_sample
+    pos, vel, types = w.pos[:n], v0[:n], w.types[:n]
+    rp, cl = oracle.neighbors(s, w.model.r_cut, pos)
+    _, forces, _ = oracle.energy_forces(w.model, w.weights, s, pos, types, rp, cl)
+    steps, t0 = 0, time.perf_counter()
+    while steps < min_steps or time.perf_counter() - t0 < budget_s:
+        pos, vel, forces, *_ = oracle.md_vv(w.model, w.weights, s, pos, vel, types, MASS, DT, 1, forces=forces)
+        steps += 1
+    dt = time.perf_counter() - t0
+    frac = n_rep_sample / w.system.n_replicas
+    return steps * frac / dt, steps, dt, oracle.num_threads()
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = synth.make_workload(CFG)
+    s = w.system
+    v0 = synth.maxwell_boltzmann(s.n_per_replica, s.n_replicas, MASS, TEMP, 4000 + CFG)
+    # size the per-step sample so that warm-up + K steps end within ~3 minutes
+    probe_rate, _, probe_t, threads = oracle_md_rate(w, v0, 8, 0.0, min_steps=max(1, min(args.warmup, 3)))
+    per_rep_s = 1.0 / (probe_rate * s.n_replicas)
+    n_sample = int(max(1, min(s.n_replicas, 150.0 / max(1, args.steps) / per_rep_s)))
+    rate, steps, secs, threads = oracle_md_rate(w, v0, n_sample, 0.0, min_steps=args.steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "evals/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": 1000.0 / rate, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": rate, "unit": "evals/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n_sample} of {s.n_replicas} replicas per step, {steps} steps in "
+                                   f"{secs:.1f} s; rate scaled to the full batch"},
+        "e2e": {"value": rate, "unit": "evals/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "utilization.gpu",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, uuid: str | None):
+        self.proc = None
+        self.uuid = uuid
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits", "-lms", "50"]
+        if self.uuid:
+            cmd[1:1] = ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        loaded = [r for r in rows if (num(r[3]) or 0) > 0] or rows
+        sm = [num(r[0]) for r in loaded if num(r[0]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in loaded:
+            for k, name in enumerate(names):
+                if r[4 + k].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": num(rows[0][1]),
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# ------------------------------------------------------------------------------ roofline
+def peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def kernel_traffic(kernel: str, src: Path):
+    """dram bytes per launch of `kernel` from the committed ncu summary, if it was taken on
+    the current source (else None)."""
+    f = ROOT / "profiles" / "traffic.txt"
+    if not f.exists():
+        return None
+    sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    for line in f.read_text().splitlines():
+        parts = dict(kv.split("=", 1) for kv in line.split()[1:] if "=" in kv)
+        if line.split() and line.split()[0] == kernel and parts.get("src") == sha and parts.get("workload") == "cfg2":
+            return float(parts["bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    from schnet_gnn_molecular_cell_b200 import Context
+
+    w = synth.make_workload(CFG)
+    s, m = w.system, w.model
+    N, R = s.n_atoms, s.n_replicas
+    v0 = synth.maxwell_boltzmann(s.n_per_replica, R, MASS, TEMP, 4000 + CFG)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    ctx = Context(m, w.weights, stream=stream)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.from_numpy(v0.copy()).to(dev)
+    types = torch.from_numpy(w.types).to(dev)
+    rp, cl = ctx.neighbors(s, pos)
+    E0 = int(cl.numel())
+    _, forces = ctx.energy_forces(s, pos, types, rp, cl)
+    forces = forces.clone()
+    ctx.reserve(s, int(1.5 * E0) + 4096)
+    energy = torch.empty(R, device=dev)
+    kin = torch.empty(R, device=dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)   # 256 MiB > L2
+
+    def step():
+        ctx.md_step(s, pos, vel, forces, types, MASS, DT, 1, energy, kin)
+
+    for k in range(args.warmup):
+        flush.fill_(float(k))
+        step()
+    ctx.sync()
+
+    uuid = None
+    try:
+        uuid = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ctx.trace(True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for k in range(args.steps):
+        flush.fill_(float(k))
+        starts[k].record(stream)
+        step()
+        ends[k].record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    trace = ctx.trace_read()
+    ctx.trace(False)
+    ctx.sync()
+    t_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
+    if world > 1:
+        t = torch.tensor([t_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.barrier()
+        t_ms = float(t.item())
+    E_last = ctx.md_edges()
+    value = world * args.steps / (t_ms / 1e3)
+
+    # dominant kernel and its roofline (algorithmic MLP flops per launch / mean launch time)
+    dom = max(trace, key=lambda k: trace[k][1])
+    launches, dom_ms = trace[dom]
+    pk, pk_kind = peaks()
+    roofline = None
+    if dom in ("edge_fwd", "edge_bwd"):
+        flops = 2.0 * (m.K * m.F + m.F * m.F) * E_last
+        achieved = flops / (dom_ms / launches / 1e3) / 1e12
+        fp32_peak = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s",
+                    "frac": achieved / fp32_peak,
+                    "traffic": kernel_traffic(dom, ROOT / "schnet_gnn_molecular_cell_b200" / "csrc" / "sn_ef_fp32.cu"),
+                    "kernel": dom, "peak_source": f"fp32 FMA: 148 SM x 128 lanes x 2 x {pk.get('sm_max_mhz', 1965.0):.0f} MHz ({pk_kind} sm_max_mhz)",
+                    "flops_per_launch": flops}
+
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+        h_pos, h_vel, h_f = pin(pos.cpu().numpy()), pin(vel.cpu().numpy()), pin(forces.cpu().numpy())
+        h_types = pin(w.types)
+        h_e = pin(np.zeros(R, np.float32))
+        h_k = pin(np.zeros(R, np.float32))
+        n_e2e = min(args.steps, 100)
+        tot = 0.0
+        for k in range(n_e2e + 2):
+            flush.fill_(float(k))
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            ctx.md_step_host(s, h_pos, h_vel, h_f, h_types, MASS, DT, 1, h_e, h_k)
+            t1 = time.perf_counter()
+            if k >= 2:
+                tot += t1 - t0
+        if world > 1:
+            t = torch.tensor([tot], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            tot = float(t.item())
+        e2e = {"value": world * n_e2e / tot, "unit": "evals/s",
+               "h2d_bytes_per_step": 3 * (3 * N * 4) + N * 4,
+               "d2h_bytes_per_step": 3 * (3 * N * 4) + 2 * R * 4,
+               "api": "sn_md_step_host (pinned host buffers; copies + step + sync timed by host clock)"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, steps, secs, threads = oracle_md_rate(w, v0, R, 10.0)
+        cpu = {"value": rate, "unit": "evals/s", "cores": threads, "kind": "oracle",
+               "sample": f"{steps} full velocity-Verlet step(s) of all {R} replicas in {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "evals/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "replicas_per_gpu": R, "beads": s.n_per_replica,
+                       "edges": E_last, "precision": "fp32 (CUDA cores)",
+                       "l2": "flushed between steps (256 MiB write, outside the timed events)",
+                       "parallelism": f"{world} rank(s), independent replica batches, no collective"},
+            "edges_per_s": value * E_last,
+            "md_steps_x_replicas_per_s": value * R,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": sum(v[0] for v in trace.values()),
+            "clocks": clocks,
+            "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0], "share": v[1] / sum(x[1] for x in trace.values())}
+                        for k, v in sorted(trace.items(), key=lambda kv: -kv[1][1])},
+        }
+        print(json.dumps(line), flush=True)
+    ctx.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,145 @@
+// Internal declarations of the B200 SchNet library: device layouts, error bits, launchers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "sn.h"
+
+namespace sn {
+
+// Kernel classes reported by the tracer (sn_trace_read).
+enum KernelKind {
+    KK_PREP = 0, KK_NB_COUNT, KK_NB_FILL, KK_SCAN, KK_CELLS, KK_PARTITION, KK_EDGE_FWD, KK_NODE_FWD,
+    KK_EDGE_BWD, KK_NODE_BWD, KK_SUMS, KK_KICK_DRIFT, KK_KICK, KK_COUNT
+};
+
+// CUDA-event timing of every kernel launch while enabled: a pair of events per launch on the
+// launching stream, read back (and reset) by sn_trace_read.
+struct Tracer {
+    bool on = false;
+    std::vector<cudaEvent_t> ev;   // 2 per record: start, end
+    std::vector<int> kinds;
+    size_t n = 0;
+    void begin(int kind, cudaStream_t s);
+    void end(cudaStream_t s);
+};
+
+inline void trace_begin(Tracer *t, int kind, cudaStream_t s)
+{
+    if (t && t->on) t->begin(kind, s);
+}
+inline void trace_end(Tracer *t, cudaStream_t s)
+{
+    if (t && t->on) t->end(s);
+}
+
+// Conditions latched on the device in ctx->d_err (bitwise OR).  Kernels that run after a
+// latched condition return without touching memory.
+enum : int {
+    ERRBIT_CAPACITY = 1,
+    ERRBIT_NONFINITE = 2,
+    ERRBIT_DEGENERATE = 4,
+};
+
+constexpr int NE = 32;        // edges per tile in the fp32 kernels
+constexpr int NA = 32;        // atoms per tile in the node kernels
+constexpr int TS = NE + 4;    // smem row stride of [feature][edge] tiles (16-byte rows)
+
+// Per-block weights in the fp32 kernel layout (device pointers into one allocation).
+// Matrices are stored [out][in] with a row stride of in+1 floats so that both "thread =
+// output" and "thread = input" sweeps read shared memory without bank conflicts.
+struct BlockW {
+    const float *W1;   // [F][KP+1], zero for k >= K
+    const float *b1;   // [F]
+    const float *W2;   // [F][F+1]
+    const float *b2;   // [F]
+    const float *U1;   // [F][F+1]
+    const float *c1;   // [F]
+    const float *U2;   // [F][F+1]
+    const float *c2;   // [F]
+};
+
+struct ReadoutW {
+    const float *R1;   // [H][F+1]
+    const float *e1;   // [H]
+    const float *R2;   // [H]
+    const float *e2;   // [1]
+};
+
+struct Geometry {
+    float box[3];      // > 0 on periodic axes
+    int periodic[3];
+};
+
+// Radial basis constants.  Centres mu_k = k * r_cut / (K - 1) are kept in double: the
+// offsets d - mu_k are formed in double and rounded once, so that the Gaussians carry no
+// error from representing d or mu_k in float (a 1e-7 A shift moves exp(-gamma x^2) by
+// 2 gamma |x| 1e-7 relative, which the cancellation in dE/dd amplifies).
+struct Basis {
+    int K, KP;
+    float r_cut, gamma;
+    double r_cut_d;
+    double mu[64];
+};
+
+// ---------------------------------------------------------------- neighbour list
+// Builds CSR (row_ptr[N+1], col[<=cap]) for n_per x n_rep atoms into caller-provided work
+// buffers.  With n_edges_host != NULL the edge count is copied back (one synchronisation) and
+// the fill pass is skipped when it exceeds cap; otherwise capacity is checked on the device
+// and an overflow is latched into d_err.
+struct NbWork {
+    float4 *pos4;      // [N]
+    int32_t *cnt;      // [N + 1]
+    int32_t *cell_of;  // [N]
+    int32_t *cell_cnt; // [ncell + 1]
+    int32_t *cell_start; // [ncell + 1]
+    int32_t *cell_atoms; // [N]
+    int64_t ncell_cap;
+};
+
+int64_t nb_cells_needed(const sn_system &sys, float r_cut, int nc[3]);
+cudaError_t launch_prep_positions(const float *pos, float4 *pos4, int64_t N, int *d_err, cudaStream_t s,
+                                  Tracer *tr);
+cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *pos4, NbWork &w,
+                             int32_t *row_ptr, int32_t *col, int64_t cap, int *d_err,
+                             int64_t *n_edges_host, cudaStream_t s, Tracer *tr);
+
+// ---------------------------------------------------------------- energy and forces
+struct EfWork {
+    const float4 *pos4;  // [N]
+    float *x;            // [T][N][F]   x^1 .. x^T
+    float *p;            // [T][N][F]   U1 h + c1 per block
+    float *h;            // [N][F]      aggregated messages of the current block
+    float *hbar;         // [N][F]      dE/dh of the current block
+    float *xbar;         // [N][F]      dE/dx of the current block (in place)
+    float *eps;          // [N]         per-atom energies
+    int32_t *part;       // [G + 1]     rows owned by each CTA of the edge kernels
+    int G;
+};
+
+struct Model {
+    int F, K, KP, T, H, n_types;
+    Basis basis;
+    const float *emb;    // [n_types][F]
+    BlockW blk[16];
+    ReadoutW ro;
+};
+
+cudaError_t launch_energy_forces(const Model &m, const sn_system &sys, const Geometry &geo,
+                                 const int32_t *types, const int32_t *row_ptr,
+                                 const int32_t *col, EfWork &w, float *energy, float *forces,
+                                 int *d_err, cudaStream_t s, Tracer *tr);
+
+// ---------------------------------------------------------------- integrator
+cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t n3, float c,
+                              float dt, int *d_err, cudaStream_t s, Tracer *tr);
+cudaError_t launch_kick(float *vel, const float *forces, int64_t n3, float c, int *d_err,
+                        cudaStream_t s, Tracer *tr);
+cudaError_t launch_replica_sums(const float *eps, const float *vel, int n_per, int n_rep,
+                                float half_m_over_kappa, float *energy, float *kinetic,
+                                int *d_err, cudaStream_t s, Tracer *tr);
+
+}  // namespace sn

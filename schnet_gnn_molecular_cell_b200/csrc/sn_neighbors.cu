@@ -1,0 +1,358 @@
+// Neighbour list on the GPU (FlashSchNet §3.2 "Building the neighbor list"; §4.3 "Index
+// construction under dynamic neighbor lists"): destination-grouped CSR with sources
+// ascending in each row.
+//
+// Membership test, float32 with every operation rounded on its own (no FMA contraction), so
+// that the list is reproducible bit for bit by any IEEE fp32 implementation:
+//   dx = x_j - x_i;  periodic axis: dx = dx - L * rint(dx / L)
+//   r2 = (dx*dx + dy*dy) + dz*dz;  edge iff r2 < r_cut*r_cut, i != j, same replica.
+//
+// Two builders:
+//   * open boundaries (or a box too small for a 3x3x3 cell stencil): all pairs of a replica,
+//     positions staged through shared memory in tiles of 128; sources come out ascending;
+//   * periodic boxes with >= 3 cells per axis: cell list (cell side >= r_cut * 1.0001), then
+//     each row is sorted by source.
+// Both run a count pass, an exclusive scan into row_ptr, and a fill pass.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "sn_internal.cuh"
+
+namespace sn {
+
+namespace {
+
+constexpr int BT = 128;   // threads per CTA / positions per shared-memory tile
+
+__device__ __forceinline__ float min_image_axis(float dx, float L)
+{
+    float q = rintf(__fdiv_rn(dx, L));
+    return __fsub_rn(dx, __fmul_rn(L, q));
+}
+
+// returns r2 of the fp32 test (see file header)
+__device__ __forceinline__ float pair_r2(float4 pi, float4 pj, const Geometry &g)
+{
+    float dx = __fsub_rn(pj.x, pi.x);
+    float dy = __fsub_rn(pj.y, pi.y);
+    float dz = __fsub_rn(pj.z, pi.z);
+    if (g.periodic[0]) dx = min_image_axis(dx, g.box[0]);
+    if (g.periodic[1]) dy = min_image_axis(dy, g.box[1]);
+    if (g.periodic[2]) dz = min_image_axis(dz, g.box[2]);
+    float r2 = __fmul_rn(dx, dx);
+    r2 = __fadd_rn(r2, __fmul_rn(dy, dy));
+    r2 = __fadd_rn(r2, __fmul_rn(dz, dz));
+    return r2;
+}
+
+__global__ void k_prep_positions(const float *__restrict__ pos, float4 *__restrict__ pos4, int64_t N,
+                                 int *__restrict__ d_err)
+{
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= N) return;
+    float x = pos[3 * i], y = pos[3 * i + 1], z = pos[3 * i + 2];
+    if (!isfinite(x) || !isfinite(y) || !isfinite(z)) {
+        atomicOr(d_err, ERRBIT_NONFINITE);
+        x = y = z = 0.0f;
+    }
+    pos4[i] = make_float4(x, y, z, 0.0f);
+}
+
+// -------------------------------------------------------------------- all pairs per replica
+// grid: (ceil(n_per / BT), n_rep); FILL = false counts, true writes sources in ascending order.
+template <bool FILL>
+__global__ void __launch_bounds__(BT) k_pairs(const float4 *__restrict__ pos4, int n_per, Geometry g, float rc2,
+                                              int32_t *__restrict__ cnt, const int32_t *__restrict__ row_ptr,
+                                              int32_t *__restrict__ col, int64_t cap, int64_t N,
+                                              int *__restrict__ d_err)
+{
+    __shared__ float4 tile[BT];
+    __shared__ int skip;
+    if (threadIdx.x == 0) {
+        // decided once per CTA: the loop below has barriers that every thread must reach
+        int k = (*((volatile int *)d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) ? 1 : 0;
+        if (FILL && !k && (int64_t)row_ptr[N] > cap) {
+            k = 1;
+            atomicOr(d_err, ERRBIT_CAPACITY);
+        }
+        skip = k;
+    }
+    __syncthreads();
+    if (skip) return;
+    const int64_t base = (int64_t)blockIdx.y * n_per;
+    const int il = blockIdx.x * BT + threadIdx.x;
+    const bool active = il < n_per;
+    const int64_t i = base + il;
+    float4 pi = active ? pos4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    int32_t c = 0;
+    int32_t w = (FILL && active) ? row_ptr[i] : 0;
+    bool degenerate = false;
+    for (int j0 = 0; j0 < n_per; j0 += BT) {
+        __syncthreads();
+        if (j0 + threadIdx.x < n_per) tile[threadIdx.x] = pos4[base + j0 + threadIdx.x];
+        __syncthreads();
+        if (!active) continue;
+        const int jn = min(BT, n_per - j0);
+        for (int q = 0; q < jn; ++q) {
+            const int jl = j0 + q;
+            if (jl == il) continue;
+            float r2 = pair_r2(pi, tile[q], g);
+            if (r2 < rc2) {
+                if (FILL) col[w++] = (int32_t)(base + jl);
+                else ++c;
+                degenerate |= (r2 == 0.0f);
+            }
+        }
+    }
+    if (!FILL && active) cnt[i] = c;
+    if (FILL && degenerate) atomicOr(d_err, ERRBIT_DEGENERATE);
+}
+
+// -------------------------------------------------------------------- cell list (periodic)
+struct CellGrid {
+    int nc[3];
+    float side[3];
+    int64_t per_rep;
+};
+
+__device__ __forceinline__ int cell_coord(float x, float L, float side, int n)
+{
+    float w = x - L * floorf(x / L);      // wrapped into [0, L] (L only through rounding)
+    int c = (int)floorf(w / side);
+    return c < 0 ? 0 : (c >= n ? n - 1 : c);
+}
+
+__global__ void k_cell_assign(const float4 *__restrict__ pos4, int64_t N, int n_per, Geometry g, CellGrid cg,
+                              int32_t *__restrict__ cell_of, int32_t *__restrict__ cell_cnt,
+                              const int *__restrict__ d_err)
+{
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= N || (*((volatile const int *)d_err) & ERRBIT_NONFINITE)) return;
+    float4 p = pos4[i];
+    int cx = cell_coord(p.x, g.box[0], cg.side[0], cg.nc[0]);
+    int cy = cell_coord(p.y, g.box[1], cg.side[1], cg.nc[1]);
+    int cz = cell_coord(p.z, g.box[2], cg.side[2], cg.nc[2]);
+    int64_t c = (i / n_per) * cg.per_rep + ((int64_t)cx * cg.nc[1] + cy) * cg.nc[2] + cz;
+    cell_of[i] = (int32_t)c;
+    atomicAdd(&cell_cnt[c], 1);
+}
+
+__global__ void k_cell_scatter(int64_t N, const int32_t *__restrict__ cell_of, int32_t *__restrict__ cursor,
+                               int32_t *__restrict__ cell_atoms, const int *__restrict__ d_err)
+{
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= N || (*((volatile const int *)d_err) & ERRBIT_NONFINITE)) return;
+    int32_t slot = atomicAdd(&cursor[cell_of[i]], 1);
+    cell_atoms[slot] = (int32_t)i;
+}
+
+template <bool FILL>
+__global__ void __launch_bounds__(BT) k_cell_pairs(const float4 *__restrict__ pos4, int64_t N, Geometry g,
+                                                   CellGrid cg, float rc2, const int32_t *__restrict__ cell_of,
+                                                   const int32_t *__restrict__ cell_start,
+                                                   const int32_t *__restrict__ cell_atoms,
+                                                   int32_t *__restrict__ cnt, const int32_t *__restrict__ row_ptr,
+                                                   int32_t *__restrict__ col, int64_t cap, int *__restrict__ d_err)
+{
+    if (*((volatile int *)d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) return;
+    if (FILL && (int64_t)row_ptr[N] > cap) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(d_err, ERRBIT_CAPACITY);
+        return;
+    }
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= N) return;
+    const float4 pi = pos4[i];
+    const int64_t c = cell_of[i];
+    const int64_t rep0 = (c / cg.per_rep) * cg.per_rep;
+    const int64_t lc = c - rep0;
+    const int cz = (int)(lc % cg.nc[2]);
+    const int cy = (int)((lc / cg.nc[2]) % cg.nc[1]);
+    const int cx = (int)(lc / ((int64_t)cg.nc[1] * cg.nc[2]));
+    int32_t n = 0;
+    const int32_t w0 = FILL ? row_ptr[i] : 0;
+    bool degenerate = false;
+    for (int ox = -1; ox <= 1; ++ox)
+        for (int oy = -1; oy <= 1; ++oy)
+            for (int oz = -1; oz <= 1; ++oz) {
+                int x = cx + ox, y = cy + oy, z = cz + oz;
+                x += (x < 0) ? cg.nc[0] : (x >= cg.nc[0] ? -cg.nc[0] : 0);
+                y += (y < 0) ? cg.nc[1] : (y >= cg.nc[1] ? -cg.nc[1] : 0);
+                z += (z < 0) ? cg.nc[2] : (z >= cg.nc[2] ? -cg.nc[2] : 0);
+                const int64_t cc = rep0 + ((int64_t)x * cg.nc[1] + y) * cg.nc[2] + z;
+                for (int32_t q = cell_start[cc]; q < cell_start[cc + 1]; ++q) {
+                    const int32_t j = cell_atoms[q];
+                    if (j == i) continue;
+                    float r2 = pair_r2(pi, pos4[j], g);
+                    if (r2 < rc2) {
+                        if (FILL) col[w0 + n] = j;
+                        ++n;
+                        degenerate |= (r2 == 0.0f);
+                    }
+                }
+            }
+    if (!FILL) {
+        cnt[i] = n;
+        return;
+    }
+    if (degenerate) atomicOr(d_err, ERRBIT_DEGENERATE);
+    // insertion sort of the row by source index (rows hold tens of entries)
+    int32_t *row = col + w0;
+    for (int32_t a = 1; a < n; ++a) {
+        int32_t v = row[a];
+        int32_t b = a - 1;
+        while (b >= 0 && row[b] > v) {
+            row[b + 1] = row[b];
+            --b;
+        }
+        row[b + 1] = v;
+    }
+}
+
+// -------------------------------------------------------------------- exclusive scan
+// One CTA of 1024 threads: out[0] = 0, out[k+1] = sum_{q<=k} in[q] for k < n.  Sums above
+// INT32_MAX latch ERRBIT_CAPACITY (a list that large cannot be indexed by int32).
+__global__ void __launch_bounds__(1024) k_scan(const int32_t *__restrict__ in, int32_t *__restrict__ out, int64_t n,
+                                               int *__restrict__ d_err)
+{
+    __shared__ long long warp_sums[32];
+    const int t = threadIdx.x;
+    const int64_t chunk = (n + 1023) / 1024;
+    const int64_t a = t * chunk;
+    const int64_t b = min(n, a + chunk);
+    long long s = 0;
+    for (int64_t q = a; q < b; ++q) s += in[q];
+    // block exclusive scan of s
+    long long v = s;
+    const int lane = t & 31, wid = t >> 5;
+    for (int o = 1; o < 32; o <<= 1) {
+        long long y = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) warp_sums[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+        long long ws = warp_sums[lane];
+        for (int o = 1; o < 32; o <<= 1) {
+            long long y = __shfl_up_sync(0xffffffffu, ws, o);
+            if (lane >= o) ws += y;
+        }
+        warp_sums[lane] = ws;
+    }
+    __syncthreads();
+    long long run = v - s + (wid > 0 ? warp_sums[wid - 1] : 0);
+    if (t == 0) out[0] = 0;
+    bool over = false;
+    for (int64_t q = a; q < b; ++q) {
+        run += in[q];
+        over |= run > 0x7fffffffLL;
+        out[q + 1] = (int32_t)(run > 0x7fffffffLL ? 0x7fffffff : run);
+    }
+    if (over) atomicOr(d_err, ERRBIT_CAPACITY);
+}
+
+__global__ void k_copy_i32(const int32_t *__restrict__ a, int32_t *__restrict__ b, int64_t n)
+{
+    int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i < n) b[i] = a[i];
+}
+
+bool use_cells(const sn_system &sys, float r_cut, int nc[3])
+{
+    for (int a = 0; a < 3; ++a) {
+        if (!(sys.box[a] > 0.0f)) return false;
+        nc[a] = (int)floor((double)sys.box[a] / ((double)r_cut * 1.0001));
+        if (nc[a] < 3) return false;
+    }
+    return true;
+}
+
+inline unsigned blocks_for(int64_t n, int bt) { return (unsigned)((n + bt - 1) / bt); }
+
+}  // namespace
+
+int64_t nb_cells_needed(const sn_system &sys, float r_cut, int nc[3])
+{
+    if (!use_cells(sys, r_cut, nc)) return 0;
+    return (int64_t)nc[0] * nc[1] * nc[2] * sys.n_replicas;
+}
+
+cudaError_t launch_prep_positions(const float *pos, float4 *pos4, int64_t N, int *d_err, cudaStream_t s,
+                                  Tracer *tr)
+{
+    if (N == 0) return cudaSuccess;
+    trace_begin(tr, KK_PREP, s);
+    k_prep_positions<<<blocks_for(N, 256), 256, 0, s>>>(pos, pos4, N, d_err);
+    trace_end(tr, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *pos4, NbWork &w,
+                             int32_t *row_ptr, int32_t *col, int64_t cap, int *d_err,
+                             int64_t *n_edges_host, cudaStream_t s, Tracer *tr)
+{
+    const int64_t N = (int64_t)sys.n_per_replica * sys.n_replicas;
+    Geometry g;
+    for (int a = 0; a < 3; ++a) {
+        g.box[a] = sys.box[a];
+        g.periodic[a] = sys.box[a] > 0.0f;
+    }
+    const float rc2 = r_cut * r_cut;
+    cudaError_t e;
+    if (N == 0) {
+        e = cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), s);
+        if (n_edges_host) *n_edges_host = 0;
+        return e;
+    }
+    int nc[3];
+    const bool cells = use_cells(sys, r_cut, nc);
+    CellGrid cg{};
+    if (cells) {
+        for (int a = 0; a < 3; ++a) {
+            cg.nc[a] = nc[a];
+            cg.side[a] = sys.box[a] / (float)nc[a];
+        }
+        cg.per_rep = (int64_t)nc[0] * nc[1] * nc[2];
+        const int64_t ncell = cg.per_rep * sys.n_replicas;
+        if (ncell > w.ncell_cap) return cudaErrorInvalidValue;
+        if ((e = cudaMemsetAsync(w.cell_cnt, 0, sizeof(int32_t) * (ncell + 1), s))) return e;
+        trace_begin(tr, KK_CELLS, s);
+        k_cell_assign<<<blocks_for(N, 256), 256, 0, s>>>(pos4, N, sys.n_per_replica, g, cg, w.cell_of, w.cell_cnt, d_err);
+        k_scan<<<1, 1024, 0, s>>>(w.cell_cnt, w.cell_start, ncell, d_err);
+        // cursor = cell_start (reuse cell_cnt as the cursor array)
+        k_copy_i32<<<blocks_for(ncell, 256), 256, 0, s>>>(w.cell_start, w.cell_cnt, ncell);
+        k_cell_scatter<<<blocks_for(N, 256), 256, 0, s>>>(N, w.cell_of, w.cell_cnt, w.cell_atoms, d_err);
+        trace_end(tr, s);
+        trace_begin(tr, KK_NB_COUNT, s);
+        k_cell_pairs<false><<<blocks_for(N, BT), BT, 0, s>>>(pos4, N, g, cg, rc2, w.cell_of, w.cell_start,
+                                                             w.cell_atoms, w.cnt, row_ptr, col, cap, d_err);
+        trace_end(tr, s);
+    } else {
+        dim3 grid(blocks_for(sys.n_per_replica, BT), sys.n_replicas);
+        trace_begin(tr, KK_NB_COUNT, s);
+        k_pairs<false><<<grid, BT, 0, s>>>(pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col, cap, N, d_err);
+        trace_end(tr, s);
+    }
+    trace_begin(tr, KK_SCAN, s);
+    k_scan<<<1, 1024, 0, s>>>(w.cnt, row_ptr, N, d_err);
+    trace_end(tr, s);
+    if ((e = cudaGetLastError())) return e;
+    if (n_edges_host) {
+        int32_t E = 0;
+        if ((e = cudaMemcpyAsync(&E, row_ptr + N, sizeof(int32_t), cudaMemcpyDeviceToHost, s))) return e;
+        if ((e = cudaStreamSynchronize(s))) return e;
+        *n_edges_host = E;
+        if (E > cap) return cudaSuccess;   // caller reports SN_ERR_CAPACITY
+    }
+    trace_begin(tr, KK_NB_FILL, s);
+    if (cells) {
+        k_cell_pairs<true><<<blocks_for(N, BT), BT, 0, s>>>(pos4, N, g, cg, rc2, w.cell_of, w.cell_start,
+                                                            w.cell_atoms, w.cnt, row_ptr, col, cap, d_err);
+    } else {
+        dim3 grid(blocks_for(sys.n_per_replica, BT), sys.n_replicas);
+        k_pairs<true><<<grid, BT, 0, s>>>(pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col, cap, N, d_err);
+    }
+    trace_end(tr, s);
+    return cudaGetLastError();
+}
+
+}  // namespace sn

@@ -1,0 +1,96 @@
+"""Velocity Verlet on the GPU (sn_md_step) vs the oracle's double-precision integrator."""
+import numpy as np
+import pytest
+
+from schnet_gnn_molecular_cell_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def _start(oracle, w, dev):
+    from schnet_gnn_molecular_cell_b200 import Context
+    s, m = w.system, w.model
+    v0 = synth.maxwell_boltzmann(s.n_per_replica, s.n_replicas, 12.0, 300.0, seed=4003)
+    ctx = Context(m, w.weights)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.from_numpy(v0.copy()).to(dev)
+    types = torch.from_numpy(w.types).to(dev)
+    rp, cl = ctx.neighbors(s, pos)
+    e0, f0 = ctx.energy_forces(s, pos, types, rp, cl)
+    return ctx, v0, pos, vel, types, f0.clone()
+
+
+@pytest.mark.parametrize("cfg,steps", [(1, 10), (2, 3), (4, 3)])
+def test_md_matches_oracle(oracle, dev, cfg, steps):
+    """Two checks.  (1) The trajectory follows the oracle's double-precision one: positions
+    are stored in fp32 (precision contract), each drift rounds r + dt v to within 2^-24 |r|,
+    so allow 1e-6 |r| + 1e-5 A; velocities and kinetic energy to 1e-4.  (2) Energy and
+    forces at the GPU's own final positions equal the oracle's at those positions, within
+    the fp32 energy/force tolerance (forces at the oracle's slightly different positions
+    differ by the Hessian times that rounding, which is not a property of the kernels)."""
+    from tests.test_gpu_parity import assert_close
+    w = synth.make_workload(cfg)
+    s = w.system
+    ctx, v0, pos, vel, types, forces = _start(oracle, w, dev)
+    energy = torch.empty(s.n_replicas, device=dev)
+    kin = torch.empty(s.n_replicas, device=dev)
+    ctx.md_step(s, pos, vel, forces, types, 12.0, 2.0, steps, energy, kin)
+    ctx.sync()
+    p_o, v_o, f_o, epot, ekin, _ = oracle.md_vv(w.model, w.weights, s, w.pos, v0, w.types, 12.0, 2.0, steps)
+    p_g = pos.cpu().numpy()
+    np.testing.assert_allclose(p_g, p_o, rtol=1e-6, atol=1e-5)
+    np.testing.assert_allclose(vel.cpu().numpy(), v_o, rtol=1e-4, atol=1e-7)
+    np.testing.assert_allclose(kin.cpu().numpy(), ekin[-1], rtol=1e-4, atol=1e-5)
+    rp, cl = oracle.neighbors(s, w.model.r_cut, p_g, "cells" if s.periodic else "brute")
+    E_o, F_o, _ = oracle.energy_forces(w.model, w.weights, s, p_g, w.types, rp, cl)
+    assert_close(energy.cpu().numpy(), E_o, "energy at final positions")
+    assert_close(forces.cpu().numpy(), F_o, "forces at final positions")
+    assert ctx.md_edges() == len(cl)
+
+
+def test_md_host_variant_equals_device(oracle, dev):
+    w = synth.make_workload(1)
+    s = w.system
+    ctx, v0, pos, vel, types, forces = _start(oracle, w, dev)
+    p_h, v_h, f_h = w.pos.copy(), v0.copy(), forces.cpu().numpy().copy()
+    e_h = np.zeros(1, np.float32)
+    k_h = np.zeros(1, np.float32)
+    energy = torch.empty(1, device=dev)
+    kin = torch.empty(1, device=dev)
+    ctx.md_step(s, pos, vel, forces, types, 12.0, 2.0, 5, energy, kin)
+    ctx.sync()
+    ctx.md_step_host(s, p_h, v_h, f_h, w.types.copy(), 12.0, 2.0, 5, e_h, k_h)
+    assert np.array_equal(p_h, pos.cpu().numpy())
+    assert np.array_equal(v_h, vel.cpu().numpy())
+    assert np.array_equal(f_h, forces.cpu().numpy())
+    assert np.array_equal(e_h, energy.cpu().numpy()) and np.array_equal(k_h, kin.cpu().numpy())
+
+
+def test_md_capacity_overflow_is_latched(dev):
+    from schnet_gnn_molecular_cell_b200 import SNError, Status
+    w = synth.make_workload(1)
+    s = w.system
+    from schnet_gnn_molecular_cell_b200 import Context
+    ctx = Context(w.model, w.weights)
+    ctx.reserve(s, 16)                       # far too small for ~576 edges
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.zeros_like(pos)
+    forces = torch.zeros_like(pos)
+    types = torch.from_numpy(w.types).to(dev)
+    e = torch.empty(1, device=dev)
+    k = torch.empty(1, device=dev)
+    ctx.md_step(s, pos, vel, forces, types, 12.0, 2.0, 2, e, k)
+    with pytest.raises(SNError) as ei:
+        ctx.sync()
+    assert ei.value.status == Status.CAPACITY
+    ctx.reserve(s, 4096)
+    ctx.md_step(s, pos, vel, forces, types, 12.0, 2.0, 1, e, k)
+    ctx.sync()

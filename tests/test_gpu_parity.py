@@ -1,0 +1,178 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Neighbour lists must match bit for bit (row_ptr and col, including order).  Energies and
+forces of the fp32 path must satisfy, per element,
+    |gpu - oracle| <= 1e-5 * max(1, RMS(oracle)) + 1e-4 * |oracle|
+i.e. 1e-4 relative / 1e-5 absolute, with the absolute part taken on the scale of the
+quantity when that scale exceeds 1 kcal/mol/A.  For all five benchmark configurations the
+force RMS is below 1, so this is exactly |err| <= 1e-5 + 1e-4 |ref|.  The stress cases with
+non-zero biases reach force RMS ~15; there fp32 rounding of the filter network alone moves
+components that cancel 1000-fold by more than an unscaled 1e-5.
+"""
+import numpy as np
+import pytest
+
+from schnet_gnn_molecular_cell_b200 import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+RTOL, ATOL = 1e-4, 1e-5
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def gpu_ctx(model, weights):
+    from schnet_gnn_molecular_cell_b200 import Context
+    return Context(model, weights)
+
+
+def to_dev(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def gpu_neighbors(ctx, system, pos, dev):
+    rp, cl = ctx.neighbors(system, to_dev(pos, dev))
+    torch.cuda.synchronize()
+    return rp.cpu().numpy(), cl.cpu().numpy()
+
+
+def assert_close(gpu, ref, what):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(gpu - ref)
+    scale = max(1.0, float(np.sqrt(np.mean(ref ** 2)))) if ref.size else 1.0
+    bound = ATOL * scale + RTOL * np.abs(ref)
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst "
+                           f"|err|={err.max():.3e} at ref={ref.flat[err.argmax()]:.4e}")
+
+
+def run_parity(oracle, w, dev, check_list=True):
+    s, m = w.system, w.model
+    ctx = gpu_ctx(m, w.weights)
+    rp_o, cl_o = oracle.neighbors(s, m.r_cut, w.pos, "cells" if s.periodic else "brute")
+    rp_g, cl_g = gpu_neighbors(ctx, s, w.pos, dev)
+    if check_list:
+        assert np.array_equal(rp_g, rp_o), "row_ptr differs"
+        assert np.array_equal(cl_g, cl_o), "col differs"
+    E_o, F_o, _ = oracle.energy_forces(m, w.weights, s, w.pos, w.types, rp_o, cl_o)
+    pos_d, types_d = to_dev(w.pos, dev), to_dev(w.types, dev)
+    E_g, F_g = ctx.energy_forces(s, pos_d, types_d, to_dev(rp_o, dev), to_dev(cl_o, dev))
+    ctx.sync()
+    assert_close(E_g.cpu().numpy(), E_o, "energy")
+    assert_close(F_g.cpu().numpy(), F_o, "forces")
+    return ctx, E_g, F_g
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 4])
+def test_config_parity(oracle, dev, cfg):
+    run_parity(oracle, synth.make_workload(cfg), dev)
+
+
+def test_config5_parity(oracle, dev):
+    """65,536 atoms, ~2.1M edges: full list bit-exact and every force component checked."""
+    run_parity(oracle, synth.make_workload(5), dev)
+
+
+CUSTOM = [
+    # (name, model, system, kind, seed, bias_std)
+    ("ragged_chains_bias", synth.ModelCfg(128, 50, 3, 20, 12.0), synth.SystemCfg(37, 5), "saw", 501, 0.2),
+    ("k32_f64_bias", synth.ModelCfg(64, 32, 2, 4, 10.0), synth.SystemCfg(45, 3), "rw", 502, 0.3),
+    ("k20_f128_T1", synth.ModelCfg(128, 20, 1, 3, 9.0, 2.5), synth.SystemCfg(70, 2), "rw", 503, 0.1),
+    ("f64_k64_T4", synth.ModelCfg(64, 64, 4, 5, 8.0, 4.0), synth.SystemCfg(33, 4), "saw", 504, 0.1),
+    ("box_aniso_bias", synth.ModelCfg(128, 50, 3, 8, 5.0), synth.SystemCfg(700, 1, (17.0, 21.5, 24.0)), "box", 505, 0.2),
+    ("box_small_fallback", synth.ModelCfg(128, 50, 2, 8, 4.0), synth.SystemCfg(90, 1, (9.0, 9.0, 9.0)), "box", 506, 0.0),
+    ("box_replicas", synth.ModelCfg(128, 50, 3, 8, 5.0), synth.SystemCfg(300, 3, (16.0, 16.0, 16.0)), "box", 507, 0.1),
+    ("one_atom_replicas", synth.ModelCfg(128, 50, 2, 8, 5.0), synth.SystemCfg(1, 7), "rw", 508, 0.2),
+]
+
+
+@pytest.mark.parametrize("name,model,system,kind,seed,bias", CUSTOM, ids=[c[0] for c in CUSTOM])
+def test_custom_parity(oracle, dev, name, model, system, kind, seed, bias):
+    run_parity(oracle, synth.make_custom(model, system, seed, kind, bias_std=bias), dev)
+
+
+def test_isolated_atoms_have_zero_force(oracle, dev):
+    m = synth.ModelCfg(128, 50, 3, 6, 5.0)
+    s = synth.SystemCfg(20, 2)
+    w = synth.make_custom(m, s, 601, "rw", bias_std=0.2)
+    pos = (np.arange(40, dtype=np.float32)[:, None] * np.array([[11.0, 0.0, 0.0]], np.float32))
+    w.pos = pos
+    ctx, E_g, F_g = run_parity(oracle, w, dev)
+    assert np.all(F_g.cpu().numpy() == 0.0)
+
+
+def test_deterministic_bitwise(dev):
+    w = synth.make_workload(4)
+    ctx = gpu_ctx(w.model, w.weights)
+    pos = to_dev(w.pos, dev)
+    types = to_dev(w.types, dev)
+    rp, cl = ctx.neighbors(w.system, pos)
+    E1, F1 = ctx.energy_forces(w.system, pos, types, rp, cl)
+    E1, F1 = E1.clone(), F1.clone()
+    E2, F2 = ctx.energy_forces(w.system, pos, types, rp, cl)
+    ctx.sync()
+    assert torch.equal(E1, E2) and torch.equal(F1, F2)
+
+
+def test_empty_system(dev):
+    m = synth.ModelCfg(128, 50, 3, 6, 5.0)
+    w = synth.weights_blob(128, 50, 3, 6, seed=1)
+    from schnet_gnn_molecular_cell_b200 import Context
+    ctx = Context(m, w)
+    s = synth.SystemCfg(0, 1)
+    pos = torch.zeros((0, 3), dtype=torch.float32, device=dev)
+    rp, cl = ctx.neighbors(s, pos)
+    assert rp.cpu().tolist() == [0] and cl.numel() == 0
+    E, F = ctx.energy_forces(s, pos, torch.zeros(0, dtype=torch.int32, device=dev), rp, cl)
+    ctx.sync()
+    assert E.cpu().tolist() == [0.0]
+
+
+def test_capacity_overflow_reports_needed_edges(oracle, dev):
+    from schnet_gnn_molecular_cell_b200 import SNError, Status
+    w = synth.make_workload(1)
+    ctx = gpu_ctx(w.model, w.weights)
+    rp_o, cl_o = oracle.neighbors(w.system, w.model.r_cut, w.pos)
+    row_ptr = torch.empty(33, dtype=torch.int32, device=dev)
+    col = torch.empty(10, dtype=torch.int32, device=dev)
+    with pytest.raises(SNError) as ei:
+        ctx.build_neighbors(w.system, to_dev(w.pos, dev), row_ptr, col)
+    assert ei.value.status == Status.CAPACITY and ei.value.needed == len(cl_o)
+    # the context stays usable
+    rp, cl = gpu_neighbors(ctx, w.system, w.pos, dev)
+    assert np.array_equal(cl, cl_o)
+
+
+def test_nonfinite_and_degenerate_are_reported(dev):
+    from schnet_gnn_molecular_cell_b200 import SNError, Status
+    w = synth.make_workload(1)
+    ctx = gpu_ctx(w.model, w.weights)
+    pos = w.pos.copy()
+    pos[5, 1] = np.nan
+    with pytest.raises(SNError) as ei:
+        ctx.neighbors(w.system, to_dev(pos, dev))
+    assert ei.value.status == Status.NONFINITE
+    pos = w.pos.copy()
+    pos[7] = pos[3]
+    with pytest.raises(SNError) as ei:
+        ctx.neighbors(w.system, to_dev(pos, dev))
+    assert ei.value.status == Status.DEGENERATE
+    rp, cl = gpu_neighbors(ctx, w.system, w.pos, dev)   # usable afterwards
+    assert len(cl) > 0
+
+
+def test_invalid_box_and_sizes(dev):
+    from schnet_gnn_molecular_cell_b200 import Context, SNError, Status
+    m = synth.ModelCfg(128, 50, 3, 8, 5.0)
+    ctx = Context(m, synth.weights_blob(128, 50, 3, 8, seed=2))
+    s = synth.SystemCfg(10, 1, (9.5, 20.0, 20.0))          # r_cut 5 >= 9.5 / 2
+    with pytest.raises(SNError) as ei:
+        ctx.neighbors(s, torch.zeros((10, 3), dtype=torch.float32, device=dev))
+    assert ei.value.status == Status.INVALID_ARG
