@@ -174,6 +174,34 @@ sn_status sn_md_step_host(sn_ctx *ctx, const sn_system *sys, float *pos_host, fl
 sn_status sn_sync(sn_ctx *ctx);
 
 /*
+ * Neighbour list without any device memory allocation.
+ *
+ * The paper has no counterpart of this entry point; it exists for callers that cannot call
+ * cudaMalloc: a host MD engine or framework that has already reserved nearly all device
+ * memory for its own pool (a raw cudaMalloc would fail or fragment it), a step loop that
+ * must not pay the implicit device synchronisation of cudaMalloc/cudaFree, or a plugin
+ * whose host application forbids allocations it does not own.  sn_build_neighbors needs a
+ * context, and creating or growing one calls cudaMalloc; this function needs no context.
+ *
+ * Output, arguments and statuses are those of sn_build_neighbors (same list, same CSR
+ * order, bit for bit), with r_cut given directly and the work enqueued on cuda_stream
+ * (a cudaStream_t, NULL = legacy default stream); it synchronises that stream once.
+ * Its work buffers are one static device array of about 2.3 MB that every GPU which loads
+ * the library keeps until the process exits.  Limits: at most SN_NOALLOC_MAX_ATOMS atoms
+ * in total and, for periodic boxes built with the cell list, at most SN_NOALLOC_MAX_CELLS
+ * cells (n_replicas x cells per box); larger systems get SN_ERR_UNSUPPORTED and nothing
+ * is launched.  The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.  All calls share
+ * the one array: calls that overlap on the GPU (different streams or host threads at the
+ * same time) race and must be serialised by the caller.
+ */
+#define SN_NOALLOC_MAX_ATOMS 65536
+#define SN_NOALLOC_MAX_CELLS 65536
+sn_status sn_build_neighbors_noalloc(const sn_system *sys, float r_cut, const float *pos_dev,
+                                     int32_t *row_ptr_dev, int32_t *col_dev, int64_t cap,
+                                     int64_t *n_edges_out, void *cuda_stream);
+
+/*
  * Kernel tracing.  While enabled, every kernel launch of the context is bracketed by a pair
  * of CUDA events on the context's stream (the events add no device work).  sn_trace_read
  * synchronises the stream, sums the elapsed times per kernel class since the last read (or

@@ -49,7 +49,8 @@ class TraceEntry(C.Structure):
 
 EXPORTS = ["sn_create", "sn_destroy", "sn_set_stream", "sn_reserve", "sn_build_neighbors",
            "sn_energy_forces", "sn_md_step", "sn_md_step_host", "sn_sync", "sn_md_edges",
-           "sn_trace_enable", "sn_trace_read", "sn_last_error", "sn_version"]
+           "sn_trace_enable", "sn_trace_read", "sn_build_neighbors_noalloc", "sn_last_error",
+           "sn_version"]
 
 _lib = None
 
@@ -79,6 +80,8 @@ def load():
     L.sn_trace_enable.restype = C.c_int
     L.sn_trace_read.argtypes = [P, C.POINTER(TraceEntry), i32]
     L.sn_trace_read.restype = i32
+    L.sn_build_neighbors_noalloc.argtypes = [C.POINTER(System), f32, P, P, P, i64, C.POINTER(i64), P]
+    L.sn_build_neighbors_noalloc.restype = C.c_int
     L.sn_last_error.argtypes = [P]
     L.sn_last_error.restype = C.c_char_p
     L.sn_version.restype = C.c_char_p
@@ -238,6 +241,28 @@ class Context:
 
     def md_edges(self) -> int:
         return int(self._L.sn_md_edges(self._h))
+
+
+def build_neighbors_noalloc(system, r_cut: float, pos, row_ptr, col, stream=None) -> int:
+    """Neighbour list through sn_build_neighbors_noalloc, for callers that cannot allocate
+    device memory: the library uses only its static scratch, the caller provides pos, row_ptr
+    [N+1] and col [cap] (int32 CUDA tensors).  Returns E; raises SNError (with .needed on
+    CAPACITY)."""
+    import torch
+    L = load()
+    _dev_check(pos, torch.float32, "pos")
+    _dev_check(row_ptr, torch.int32, "row_ptr")
+    _dev_check(col, torch.int32, "col")
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    ne = C.c_int64(0)
+    st = L.sn_build_neighbors_noalloc(C.byref(system_struct(system)), float(r_cut), _ptr(pos), _ptr(row_ptr),
+                                      _ptr(col), col.numel(), C.byref(ne), C.c_void_p(stream.cuda_stream))
+    if st != 0:
+        err = SNError(st, "sn_build_neighbors_noalloc failed")
+        err.needed = ne.value
+        raise err
+    return ne.value
 
 
 def version() -> str:
