@@ -49,12 +49,21 @@ typedef enum {
     SN_ERR_DEGENERATE = 4,    /* two atoms of one replica at distance 0 (direction undefined) */
     SN_ERR_CUDA = 5,          /* a CUDA runtime call failed; message in sn_last_error      */
     SN_ERR_UNSUPPORTED = 6,   /* model size outside what the kernels are built for         */
-    SN_ERR_NOMEM = 7          /* device or host allocation failed                          */
+    SN_ERR_NOMEM = 7,         /* device or host allocation failed                          */
+    SN_ERR_TIMEOUT = 8        /* a kernel gave up waiting for its own tensor-core work      */
 } sn_status;
 
-/* Arithmetic of the filter and update networks. */
+/* Arithmetic of the filter network (update and readout networks are fp32 in all modes).
+ *  SN_PREC_FP32: fp32 on CUDA cores.
+ *  SN_PREC_FP16: fp16 operands on the tensor cores (tcgen05), fp32 accumulation in TMEM --
+ *                the W16A16 precision of FlashSchNet §4.4 (per-tensor, no calibration).
+ *  SN_PREC_TC32: fp32-accurate on the tensor cores: every operand split into two fp16
+ *                terms, products accumulated as hi*hi + hi*lo + lo*hi (3 MMAs).
+ * The tensor-core modes need F = 128. */
 enum {
-    SN_PREC_FP32 = 0          /* fp32 operands, fp32 accumulation (CUDA cores)             */
+    SN_PREC_FP32 = 0,
+    SN_PREC_FP16 = 1,
+    SN_PREC_TC32 = 2
 };
 
 /* Model hyper-parameters.  Supported: F in {64, 128}, 2 <= K <= 64, T >= 1, n_types >= 1. */

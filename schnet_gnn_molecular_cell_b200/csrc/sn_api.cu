@@ -30,6 +30,7 @@ struct sn_ctx {
     int device = 0;
     int n_sm = 148;
     float *d_weights = nullptr;
+    uint16_t *d_tcw = nullptr;         // fp16 hi/lo filter weights for the tensor-core modes
     sn::Model model{};
     int *d_err = nullptr;
     int32_t *h_err = nullptr;          // pinned
@@ -219,6 +220,7 @@ sn_status status_from_bits(sn_ctx *ctx, int bits)
     if (bits & sn::ERRBIT_CAPACITY) return fail(ctx, SN_ERR_CAPACITY, "neighbour list exceeded the edge capacity");
     if (bits & sn::ERRBIT_NONFINITE) return fail(ctx, SN_ERR_NONFINITE, "non-finite position");
     if (bits & sn::ERRBIT_DEGENERATE) return fail(ctx, SN_ERR_DEGENERATE, "two atoms at distance 0");
+    if (bits & sn::ERRBIT_TIMEOUT) return fail(ctx, SN_ERR_TIMEOUT, "a kernel timed out waiting for its tensor-core work");
     return SN_OK;
 }
 
@@ -276,7 +278,10 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
     const int F = cfg->F, K = cfg->K, T = cfg->T, NT = cfg->n_types;
     if (!(cfg->r_cut > 0.0f) || isinf(cfg->r_cut) || !(cfg->gamma > 0.0f) || NT < 1 || K < 2 || T < 1 || F < 2)
         return SN_ERR_INVALID_ARG;
-    if (!(F == 64 || F == 128) || K > 64 || T > MAX_T || cfg->precision != SN_PREC_FP32) return SN_ERR_UNSUPPORTED;
+    if (!(F == 64 || F == 128) || K > 64 || T > MAX_T) return SN_ERR_UNSUPPORTED;
+    if (cfg->precision != SN_PREC_FP32 && cfg->precision != SN_PREC_FP16 && cfg->precision != SN_PREC_TC32)
+        return SN_ERR_INVALID_ARG;
+    if (cfg->precision != SN_PREC_FP32 && F != 128) return SN_ERR_UNSUPPORTED;
     const int H = F / 2;
     const int64_t per_block = (int64_t)F * K + F + 3 * ((int64_t)F * F + F);
     const int64_t expect = (int64_t)NT * F + T * per_block + (int64_t)H * F + H + H + 1;
@@ -333,7 +338,23 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
         }
     }
 
+    // fp16 hi/lo copies of W1 and W2 in the tensor-core operand layout (per block: W1h W1l W2h W2l)
+    std::vector<uint16_t> tcw;
+    const size_t n_w1 = (size_t)F * KP, n_w2 = (size_t)F * F, per_tc = 2 * n_w1 + 2 * n_w2;
+    if (cfg->precision != SN_PREC_FP32) {
+        tcw.assign(per_tc * T, 0);
+        for (int t = 0; t < T; ++t) {
+            const float *blk = weights_host + (int64_t)NT * F + t * per_block;
+            uint16_t *o = tcw.data() + per_tc * t;
+            sn::tc_pack_matrix(blk, F, K, KP, o, o + n_w1);
+            sn::tc_pack_matrix(blk + (int64_t)F * K + F, F, F, F, o + 2 * n_w1, o + 2 * n_w1 + n_w2);
+        }
+    }
+
     cudaError_t e = cudaMalloc(&ctx->d_weights, sizeof(float) * pk.buf.size());
+    if (e == cudaSuccess && !tcw.empty()) e = cudaMalloc(&ctx->d_tcw, sizeof(uint16_t) * tcw.size());
+    if (e == cudaSuccess && !tcw.empty())
+        e = cudaMemcpy(ctx->d_tcw, tcw.data(), sizeof(uint16_t) * tcw.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(ctx->d_weights, pk.buf.data(), sizeof(float) * pk.buf.size(), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMalloc(&ctx->d_err, sizeof(int));
     if (e == cudaSuccess) e = cudaMemset(ctx->d_err, 0, sizeof(int));
@@ -351,6 +372,7 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
     m.T = T;
     m.H = H;
     m.n_types = NT;
+    m.precision = cfg->precision;
     m.basis.K = K;
     m.basis.KP = KP;
     m.basis.r_cut = cfg->r_cut;
@@ -367,6 +389,13 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
         m.blk[t].c1 = W + o_blk[t][5];
         m.blk[t].U2 = W + o_blk[t][6];
         m.blk[t].c2 = W + o_blk[t][7];
+        if (ctx->d_tcw) {
+            const uint16_t *o = ctx->d_tcw + per_tc * t;
+            m.blk[t].W1h = o;
+            m.blk[t].W1l = o + n_w1;
+            m.blk[t].W2h = o + 2 * n_w1;
+            m.blk[t].W2l = o + 2 * n_w1 + n_w2;
+        }
     }
     m.ro.R1 = W + o_R1;
     m.ro.e1 = W + o_e1;
@@ -387,6 +416,7 @@ sn_status sn_destroy(sn_ctx *ctx)
     for (DevBuf *b : bufs) release(*b);
     for (cudaEvent_t ev : ctx->tracer.ev) cudaEventDestroy(ev);
     if (ctx->d_weights) cudaFree(ctx->d_weights);
+    if (ctx->d_tcw) cudaFree(ctx->d_tcw);
     if (ctx->d_err) cudaFree(ctx->d_err);
     if (ctx->h_err) cudaFreeHost(ctx->h_err);
     delete ctx;

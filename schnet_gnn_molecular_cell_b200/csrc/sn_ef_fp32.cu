@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(F) k_edge_fwd(EdgeArgs A)
     __shared__ int skip;
 
     const int f = threadIdx.x;
-    if (f == 0) skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) != 0;
+    if (f == 0) skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     copy_f4(sW1, A.w.W1, S::W1, f, F);
     copy_f4(sW2, A.w.W2, S::W2, f, F);
     const float b1f = A.w.b1[f], b2f = A.w.b2[f];
@@ -270,7 +270,7 @@ __global__ void __launch_bounds__(F) k_edge_bwd(EdgeArgs A)
     __shared__ int skip;
 
     const int f = threadIdx.x;
-    if (f == 0) skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) != 0;
+    if (f == 0) skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     copy_f4(sW1, A.w.W1, S::W1, f, F);
     copy_f4(sW2, A.w.W2, S::W2, f, F);
     const float b1f = A.w.b1[f], b2f = A.w.b2[f];
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(F) k_node_fwd(NodeArgs A)
     __shared__ int skip;
 
     const int f = threadIdx.x;
-    if (f == 0) skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) != 0;
+    if (f == 0) skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     copy_f4(sU1, A.w.U1, S::U, f, F);
     copy_f4(sU2, A.w.U2, S::U, f, F);
     if (LAST) copy_f4(sR1, A.ro.R1, S::R, f, F);
@@ -528,7 +528,7 @@ __global__ void __launch_bounds__(F) k_node_bwd(NodeArgs A)
     __shared__ int skip;
 
     const int f = threadIdx.x;
-    if (f == 0) skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) != 0;
+    if (f == 0) skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     copy_f4(sU1, A.w.U1, S::U, f, F);
     copy_f4(sU2, A.w.U2, S::U, f, F);
     __syncthreads();
@@ -563,6 +563,34 @@ __global__ void k_partition(const int32_t *__restrict__ row_ptr, int64_t N, int 
         else lo = mid + 1;
     }
     part[c] = (int32_t)lo;
+}
+
+EdgeTcArgs tc_args(const EdgeArgs &a, const BlockW &bw, int *d_err)
+{
+    EdgeTcArgs t{};
+    t.pos4 = a.pos4;
+    t.types = a.types;
+    t.row_ptr = a.row_ptr;
+    t.col = a.col;
+    t.part = a.part;
+    t.emb = a.emb;
+    t.X = a.X;
+    t.H = a.H;
+    t.Hbar = a.Hbar;
+    t.Xbar = a.Xbar;
+    t.forces = a.forces;
+    t.N = a.N;
+    t.geo = a.geo;
+    t.basis = a.basis;
+    t.W1h = bw.W1h;
+    t.W1l = bw.W1l;
+    t.W2h = bw.W2h;
+    t.W2l = bw.W2l;
+    t.b1 = bw.b1;
+    t.b2 = bw.b2;
+    t.t = a.t;
+    t.d_err = d_err;
+    return t;
 }
 
 template <typename Kern>
@@ -630,7 +658,8 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
         ea.w = m.blk[t];
         ea.t = t;
         trace_begin(tr, KK_EDGE_FWD, s);
-        k_edge_fwd<F, KP><<<w.G, F, fwd_bytes, s>>>(ea);
+        if (m.precision == SN_PREC_FP32) k_edge_fwd<F, KP><<<w.G, F, fwd_bytes, s>>>(ea);
+        else if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err), KP, m.precision == SN_PREC_TC32, false, w.G, s))) return e;
         trace_end(tr, s);
         na.w = m.blk[t];
         na.t = t;
@@ -643,7 +672,8 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
         ea.w = m.blk[t];
         ea.t = t;
         trace_begin(tr, KK_EDGE_BWD, s);
-        k_edge_bwd<F, KP><<<w.G, F, bwd_bytes, s>>>(ea);
+        if (m.precision == SN_PREC_FP32) k_edge_bwd<F, KP><<<w.G, F, bwd_bytes, s>>>(ea);
+        else if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err), KP, m.precision == SN_PREC_TC32, true, w.G, s))) return e;
         trace_end(tr, s);
         if (t > 0) {
             na.w = m.blk[t - 1];

@@ -1,0 +1,699 @@
+// Edge kernels on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
+//
+// The filter network of every edge tile is a dense contraction (FlashSchNet §3.3 "Mixed
+// precision and Tensor Cores", §4.4): per tile of TE = 128 edges
+//   forward   D_A[f][n] = W1[f][:] . bt[n][:]          (M = F = 128, N = 128, K = K_P)
+//             D_W[f][n] = W2[f][:] . s[n][:]           (M = 128, N = 128, K = F)
+//   backward  D_S[i][n] = W2[:][i] . wbar[n][:]        (W2^T, M = 128, N = 128, K = F)
+//             D_G[n][k] = abar[n][:] . W1[:][k]        (edges on M: M = 128, N = K_P, K = F)
+// with fp16 operands in shared memory and fp32 accumulation in TMEM (the pages' W16A16 for
+// MLPs with fp32 accumulation, §4.1).  SPLIT adds an fp32-accurate mode: every operand x is
+// split into hi = fp16(x) and lo = fp16(x - hi), and each product is accumulated as
+// hi*hi + hi*lo + lo*hi (three MMAs into the same accumulator, ~22 significant bits).
+//
+// One CTA (one warpgroup of 128 threads) per SM owns whole destination rows (as the fp32
+// kernels do) and walks their edges tile by tile.  Thread t is TMEM lane t: for the
+// feature-major accumulators it is feature f = t, for D_G it is edge n = t.  The elementwise
+// work between the MMAs (Gaussians, ssp, gathers, segment sums) runs on the CUDA cores.
+//
+// Shared-memory operand layout: no swizzle, 8 x 16-byte "core matrices".  An element (r, c)
+// of a matrix whose contiguous 8-element runs go along c sits at
+//   (r % 8) * 16 + (r / 8) * SBO + (c % 8) * 2 + (c / 8) * LBO   bytes.
+// The same bytes read as K-major for one GEMM read as MN-major for its transpose with LBO and
+// SBO exchanged, so each weight matrix is stored once and serves forward and backward.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "sn_internal.cuh"
+
+namespace sn {
+
+namespace {
+
+constexpr int TE = 128;          // edges per tile
+constexpr int NT = 128;          // threads per CTA
+constexpr int FF = 128;          // feature width supported by these kernels
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_A = 0, COL_W = 128, COL_S = 256, COL_G = 384;
+constexpr float LN2F = 0.693147180559945309f;
+
+// ------------------------------------------------------------------ PTX wrappers (sm_100a)
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t holder, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t mbar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mbar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    return ok;
+}
+
+// This lane's 32 consecutive 32-bit TMEM columns starting at taddr (warp w reads lanes 32w..).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor, no swizzle (layout type 0), version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+// Instruction descriptor for kind::f16: fp16 A and B, fp32 D, dense.
+constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major)
+{
+    return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+// ------------------------------------------------------------------ helpers
+__device__ __forceinline__ float featv(int t, const float *__restrict__ X, const float *__restrict__ emb,
+                                       const int32_t *__restrict__ types, int64_t N, int j, int f)
+{
+    if (t == 0) return __ldg(emb + (int64_t)__ldg(types + j) * FF + f);
+    return __ldg(X + ((int64_t)(t - 1) * N + j) * FF + f);
+}
+
+__device__ __forceinline__ int row_of_edge(const int32_t *__restrict__ row_ptr, int i0, int i1, int e)
+{
+    int lo = i0, hi = i1 - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (__ldg(row_ptr + mid) <= e) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ uint32_t pack_h2(__half a, __half b)
+{
+    return (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
+}
+
+// 8 values -> one 16-byte fp16 run (hi) and, for SPLIT, the run of residuals (lo)
+template <bool SPLIT>
+__device__ __forceinline__ void store8(unsigned char *hi, unsigned char *lo, uint32_t off, const float *v)
+{
+    __half h[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) h[q] = __float2half_rn(v[q]);
+    *reinterpret_cast<uint4 *>(hi + off) =
+        make_uint4(pack_h2(h[0], h[1]), pack_h2(h[2], h[3]), pack_h2(h[4], h[5]), pack_h2(h[6], h[7]));
+    if (SPLIT) {
+        __half l[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) l[q] = __float2half_rn(v[q] - __half2float(h[q]));
+        *reinterpret_cast<uint4 *>(lo + off) =
+            make_uint4(pack_h2(l[0], l[1]), pack_h2(l[2], l[3]), pack_h2(l[4], l[5]), pack_h2(l[6], l[7]));
+    }
+}
+
+// Activation tile T[n][f] (edges n contiguous in 16-byte runs): element (n, f) at
+// (n % 8) * 2 + (n / 8) * 2048 + (f % 8) * 16 + (f / 8) * 128.  Thread f stores edges
+// n0 .. n0+31 of its feature.
+template <bool SPLIT>
+__device__ __forceinline__ void store_tile_col(unsigned char *Th, unsigned char *Tl, int f, int n0, const float (&v)[32])
+{
+    const uint32_t base = (uint32_t)((f & 7) * 16 + (f >> 3) * 128);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) store8<SPLIT>(Th, Tl, base + (uint32_t)(((n0 >> 3) + g) * 2048), v + 8 * g);
+}
+
+// Bounded wait for the MMAs committed to mbar; every thread calls it at the same point.  On
+// a time-out (never expected: nothing here waits on another agent) the error bit is set and
+// all threads return false together.
+__device__ __forceinline__ bool wait_mma(uint32_t mbar, uint32_t &phase, int *d_err)
+{
+    const long long t0 = clock64();
+    int ok = 0;
+    for (;;) {
+        if (mbar_try_wait(mbar, phase)) {
+            ok = 1;
+            break;
+        }
+        if (clock64() - t0 > (1ll << 33)) break;
+    }
+    phase ^= 1u;
+    ok = __syncthreads_and(ok);
+    if (!ok && threadIdx.x == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
+    tc_fence_after();
+    return ok != 0;
+}
+
+// Shared-memory plan of both kernels (bytes).
+template <int KP, bool SPLIT>
+struct TcSmem {
+    static constexpr int NS = SPLIT ? 2 : 1;
+    static constexpr uint32_t W1B = FF * KP * 2;        // one fp16 copy of W1
+    static constexpr uint32_t W2B = FF * FF * 2;
+    static constexpr uint32_t BB = TE * KP * 2;         // basis tile
+    static constexpr uint32_t TB = TE * FF * 2;         // activation tile
+    static constexpr uint32_t W1 = 0;
+    static constexpr uint32_t W2 = W1 + NS * W1B;
+    static constexpr uint32_t B = W2 + NS * W2B;
+    static constexpr uint32_t T = B + NS * BB;
+    static constexpr uint32_t META = T + NS * TB;       // src, dst (int), d (double), u[3], fv[3] (float)
+    static constexpr uint32_t SRC = META;
+    static constexpr uint32_t DST = SRC + 4 * TE;
+    static constexpr uint32_t DIST = DST + 4 * TE;
+    static constexpr uint32_t UVEC = DIST + 8 * TE;
+    static constexpr uint32_t FV = UVEC + 12 * TE;
+    static constexpr uint32_t MBAR = FV + 12 * TE;
+    static constexpr uint32_t HOLD = MBAR + 8;
+    static constexpr uint32_t USED = HOLD + 16;
+    // at least 116 KB so that no two CTAs share an SM (each allocates all 512 TMEM columns)
+    static constexpr uint32_t BYTES = USED > 116 * 1024 ? USED : 116 * 1024;
+    static constexpr uint32_t SW1 = (KP / 8) * 128;     // 8-row group stride of W1 and of the basis tile
+};
+
+}  // namespace
+
+namespace {
+
+template <bool ACCURATE>
+__device__ __forceinline__ float ssp_t(float x)
+{
+    return fmaxf(x, 0.0f) + log1pf(ACCURATE ? expf(-fabsf(x)) : __expf(-fabsf(x))) - LN2F;
+}
+template <bool ACCURATE>
+__device__ __forceinline__ float sigmoid_t(float x)
+{
+    return ACCURATE ? 1.0f / (1.0f + expf(-x)) : __fdividef(1.0f, 1.0f + __expf(-x));
+}
+
+__device__ __forceinline__ void copy_to_smem(unsigned char *dst, const void *src, uint32_t bytes)
+{
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+    for (uint32_t q = threadIdx.x; q < bytes / 16; q += NT) d[q] = __ldg(s + q);
+}
+
+// Edge metadata and the basis row of edge n = threadIdx.x: u = r_i - r_j and d in double
+// (minimum image on periodic axes), unit vector, and bt_k = exp(-gamma (d - mu_k)^2) C(d) as
+// fp16 (hi/lo) in the basis tile; zero for k >= K and for padding edges n >= ne.
+template <int KP, bool SPLIT>
+__device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char *sm, int i0, int i1, int ts, int ne)
+{
+    using S = TcSmem<KP, SPLIT>;
+    const int n = threadIdx.x;
+    int *sSrc = reinterpret_cast<int *>(sm + S::SRC);
+    int *sDst = reinterpret_cast<int *>(sm + S::DST);
+    double *sDist = reinterpret_cast<double *>(sm + S::DIST);
+    float *sU = reinterpret_cast<float *>(sm + S::UVEC);
+    double d = 0.0;
+    if (n < ne) {
+        const int e = ts + n;
+        const int j = __ldg(A.col + e);
+        const int i = row_of_edge(A.row_ptr, i0, i1, e);
+        const float4 ri = A.pos4[i], rj = A.pos4[j];
+        double dx = (double)ri.x - (double)rj.x, dy = (double)ri.y - (double)rj.y, dz = (double)ri.z - (double)rj.z;
+        if (A.geo.periodic[0]) dx -= (double)A.geo.box[0] * rint(dx / (double)A.geo.box[0]);
+        if (A.geo.periodic[1]) dy -= (double)A.geo.box[1] * rint(dy / (double)A.geo.box[1]);
+        if (A.geo.periodic[2]) dz -= (double)A.geo.box[2] * rint(dz / (double)A.geo.box[2]);
+        d = sqrt(dx * dx + dy * dy + dz * dz);
+        sSrc[n] = j;
+        sDst[n] = i;
+        sDist[n] = d;
+        sU[3 * n] = (float)(dx / d);
+        sU[3 * n + 1] = (float)(dy / d);
+        sU[3 * n + 2] = (float)(dz / d);
+    } else {
+        sSrc[n] = -1;
+        sDst[n] = -1;
+        sDist[n] = 0.0;
+    }
+    const float C = 0.5f * (cospif((float)(d / A.basis.r_cut_d)) + 1.0f);
+    unsigned char *Bh = sm + S::B;
+    unsigned char *Bl = Bh + S::BB;
+    const uint32_t row = (uint32_t)((n & 7) * 16 + (n >> 3) * S::SW1);
+#pragma unroll
+    for (int q = 0; q < KP / 8; ++q) {
+        float v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const int k = 8 * q + c;
+            float b = 0.0f;
+            if (n < ne && k < A.basis.K) {
+                const float x = (float)(d - A.basis.mu[k]);
+                b = expf(-A.basis.gamma * x * x) * C;
+            }
+            v[c] = b;
+        }
+        store8<SPLIT>(Bh, Bl, row + (uint32_t)q * 128, v);
+    }
+}
+
+// D_A[f][n] = sum_k W1[f][k] bt[n][k]
+template <int KP, bool SPLIT>
+__device__ __forceinline__ void issue_mma1(unsigned char *sm, uint32_t d)
+{
+    using S = TcSmem<KP, SPLIT>;
+    constexpr uint32_t ID = idesc_f16(128, TE, 0, 0);
+    const uint32_t wh = smem_u32(sm + S::W1), wl = wh + S::W1B;
+    const uint32_t bh = smem_u32(sm + S::B), bl = bh + S::BB;
+#pragma unroll
+    for (int j = 0; j < KP / 16; ++j) {
+        const uint32_t o = (uint32_t)j * 256;
+        mma_f16(d, sdesc(wh + o, 128, S::SW1), sdesc(bh + o, 128, S::SW1), ID, j > 0);
+        if (SPLIT) {
+            mma_f16(d, sdesc(wh + o, 128, S::SW1), sdesc(bl + o, 128, S::SW1), ID, 1);
+            mma_f16(d, sdesc(wl + o, 128, S::SW1), sdesc(bh + o, 128, S::SW1), ID, 1);
+        }
+    }
+}
+
+// TRANS = false: D[o][n] = sum_i W2[o][i] T[n][i]   (forward filter layer 2)
+// TRANS = true : D[i][n] = sum_o W2[o][i] T[n][o]   (backward through layer 2)
+template <int KP, bool SPLIT, bool TRANS>
+__device__ __forceinline__ void issue_mma_w2(unsigned char *sm, uint32_t d)
+{
+    using S = TcSmem<KP, SPLIT>;
+    constexpr uint32_t ID = idesc_f16(128, TE, TRANS ? 1 : 0, 1);
+    const uint32_t wh = smem_u32(sm + S::W2), wl = wh + S::W2B;
+    const uint32_t th = smem_u32(sm + S::T), tl = th + S::TB;
+    const uint32_t a_lbo = TRANS ? 2048 : 128, a_sbo = TRANS ? 128 : 2048, a_step = TRANS ? 4096 : 256;
+#pragma unroll
+    for (int j = 0; j < FF / 16; ++j) {
+        const uint32_t oa = (uint32_t)j * a_step, ob = (uint32_t)j * 256;
+        mma_f16(d, sdesc(wh + oa, a_lbo, a_sbo), sdesc(th + ob, 128, 2048), ID, j > 0);
+        if (SPLIT) {
+            mma_f16(d, sdesc(wh + oa, a_lbo, a_sbo), sdesc(tl + ob, 128, 2048), ID, 1);
+            mma_f16(d, sdesc(wl + oa, a_lbo, a_sbo), sdesc(th + ob, 128, 2048), ID, 1);
+        }
+    }
+}
+
+// D_G[n][k] = sum_f abar[n][f] W1[f][k]   (edges on M)
+template <int KP, bool SPLIT>
+__device__ __forceinline__ void issue_mma4(unsigned char *sm, uint32_t d)
+{
+    using S = TcSmem<KP, SPLIT>;
+    constexpr uint32_t ID = idesc_f16(128, KP, 1, 1);
+    const uint32_t wh = smem_u32(sm + S::W1), wl = wh + S::W1B;
+    const uint32_t th = smem_u32(sm + S::T), tl = th + S::TB;
+#pragma unroll
+    for (int j = 0; j < FF / 16; ++j) {
+        const uint32_t oa = (uint32_t)j * 256, ob = (uint32_t)j * 2 * S::SW1;
+        mma_f16(d, sdesc(th + oa, 128, 2048), sdesc(wh + ob, S::SW1, 128), ID, j > 0);
+        if (SPLIT) {
+            mma_f16(d, sdesc(tl + oa, 128, 2048), sdesc(wh + ob, S::SW1, 128), ID, 1);
+            mma_f16(d, sdesc(th + oa, 128, 2048), sdesc(wl + ob, S::SW1, 128), ID, 1);
+        }
+    }
+}
+
+// Common kernel set-up: weights to shared memory, mbarrier, TMEM allocation.
+template <int KP, bool SPLIT>
+__device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm, int &skip)
+{
+    using S = TcSmem<KP, SPLIT>;
+    const int warp = threadIdx.x >> 5;
+    copy_to_smem(sm + S::W1, A.W1h, S::W1B);
+    copy_to_smem(sm + S::W2, A.W2h, S::W2B);
+    if (SPLIT) {
+        copy_to_smem(sm + S::W1 + S::W1B, A.W1l, S::W1B);
+        copy_to_smem(sm + S::W2 + S::W2B, A.W2l, S::W2B);
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(sm + S::MBAR), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
+    }
+    if (warp == 0) tmem_alloc(smem_u32(sm + S::HOLD), TMEM_COLS);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
+}
+
+template <int KP, bool SPLIT>
+__device__ __forceinline__ void teardown(uint32_t tmem)
+{
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+template <int KP, bool SPLIT>
+__global__ void __launch_bounds__(NT, 1) k_edge_fwd_tc(EdgeTcArgs A)
+{
+    using S = TcSmem<KP, SPLIT>;
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ int skip;
+    const int f = threadIdx.x, warp = f >> 5;
+    const uint32_t tmem = setup<KP, SPLIT>(A, sm, skip);
+    const uint32_t mbar = smem_u32(sm + S::MBAR);
+    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+    const int i0 = A.part[blockIdx.x], i1 = A.part[blockIdx.x + 1];
+    if (!skip && i0 < i1) {
+        const int e0 = A.row_ptr[i0], e1 = A.row_ptr[i1];
+        const float b1f = A.b1[f], b2f = A.b2[f];
+        const int *sSrc = reinterpret_cast<const int *>(sm + S::SRC);
+        const int *sDst = reinterpret_cast<const int *>(sm + S::DST);
+        unsigned char *Th = sm + S::T, *Tl = Th + S::TB;
+        uint32_t phase = 0;
+        int cur = i0;
+        float hacc = 0.0f;
+        bool ok = true;
+        for (int ts = e0; ts < e1 && ok; ts += TE) {
+            const int ne = min(TE, e1 - ts);
+            tile_prologue<KP, SPLIT>(A, sm, i0, i1, ts, ne);
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (f == 0) {
+                tc_fence_after();
+                issue_mma1<KP, SPLIT>(sm, tmem + COL_A);
+                mma_commit(mbar);
+            }
+            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+            // s = ssp(a + b1) into the activation tile
+#pragma unroll 1
+            for (int c = 0; c < TE / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane + COL_A + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) v[q] = ssp_t<SPLIT>(v[q] + b1f);
+                store_tile_col<SPLIT>(Th, Tl, f, 32 * c, v);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (f == 0) {
+                tc_fence_after();
+                issue_mma_w2<KP, SPLIT, false>(sm, tmem + COL_W);
+                mma_commit(mbar);
+            }
+            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+            // h_i += x_src (.) (w + b2), segment sums per destination row
+#pragma unroll 1
+            for (int c = 0; c < TE / 32; ++c) {
+                if (32 * c >= ne) break;
+                float v[32], xs[32];
+                tmem_ld32(tmem + lane + COL_W + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int n = 32 * c + q;
+                    xs[q] = n < ne ? featv(A.t, A.X, A.emb, A.types, A.N, sSrc[n], f) : 0.0f;
+                }
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int n = 32 * c + q;
+                    if (n < ne) {
+                        const int i = sDst[n];
+                        if (i != cur) {
+                            A.H[(int64_t)cur * FF + f] = hacc;
+                            for (int r = cur + 1; r < i; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
+                            hacc = 0.0f;
+                            cur = i;
+                        }
+                        hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+        }
+        if (ok) {
+            A.H[(int64_t)cur * FF + f] = hacc;
+            for (int r = cur + 1; r < i1; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
+        }
+    }
+    teardown<KP, SPLIT>(tmem);
+}
+
+// Backward of one interaction block over the CTA's rows (see sn_ef_fp32.cu for the algebra):
+// recompute a = W1 bt + b1 and w = W2 ssp(a) + b2; xbar_i += sum_j hbar_j (.) w_ij;
+// wbar = x_j (.) hbar_i + x_i (.) hbar_j; sbar = W2^T wbar; abar = sbar (.) sigma(a);
+// btbar = W1^T abar (edges on M, one TMEM lane per edge); dbar = btbar . d(bt)/dd;
+// F_i -= dbar * u_ij / d_ij, accumulated by the row's owner only.
+template <int KP, bool SPLIT>
+__global__ void __launch_bounds__(NT, 1) k_edge_bwd_tc(EdgeTcArgs A)
+{
+    using S = TcSmem<KP, SPLIT>;
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ int skip;
+    const int f = threadIdx.x, warp = f >> 5;
+    const uint32_t tmem = setup<KP, SPLIT>(A, sm, skip);
+    const uint32_t mbar = smem_u32(sm + S::MBAR);
+    const uint32_t lane = (uint32_t)(warp * 32) << 16;
+    const int i0 = A.part[blockIdx.x], i1 = A.part[blockIdx.x + 1];
+    if (!skip && i0 < i1) {
+        const int e0 = A.row_ptr[i0], e1 = A.row_ptr[i1];
+        const float b1f = A.b1[f], b2f = A.b2[f];
+        const int *sSrc = reinterpret_cast<const int *>(sm + S::SRC);
+        const int *sDst = reinterpret_cast<const int *>(sm + S::DST);
+        const double *sDist = reinterpret_cast<const double *>(sm + S::DIST);
+        const float *sU = reinterpret_cast<const float *>(sm + S::UVEC);
+        float *sFv = reinterpret_cast<float *>(sm + S::FV);
+        unsigned char *Th = sm + S::T, *Tl = Th + S::TB;
+        uint32_t phase = 0;
+        int cur = -1;
+        float xbacc = 0.0f, hbi = 0.0f, xi = 0.0f;
+        bool ok = true;
+        for (int ts = e0; ts < e1 && ok; ts += TE) {
+            const int ne = min(TE, e1 - ts);
+            tile_prologue<KP, SPLIT>(A, sm, i0, i1, ts, ne);
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (f == 0) {
+                tc_fence_after();
+                issue_mma1<KP, SPLIT>(sm, tmem + COL_A);
+                mma_commit(mbar);
+            }
+            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+#pragma unroll 1
+            for (int c = 0; c < TE / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane + COL_A + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) v[q] = ssp_t<SPLIT>(v[q] + b1f);
+                store_tile_col<SPLIT>(Th, Tl, f, 32 * c, v);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (f == 0) {
+                tc_fence_after();
+                issue_mma_w2<KP, SPLIT, false>(sm, tmem + COL_W);
+                mma_commit(mbar);
+            }
+            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+            // xbar and wbar (the activation tile is free: the MMA that read s has completed)
+#pragma unroll 1
+            for (int c = 0; c < TE / 32; ++c) {
+                float w[32], hb[32], xj[32];
+                tmem_ld32(tmem + lane + COL_W + 32 * c, w);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int n = 32 * c + q;
+                    if (n < ne) {
+                        const int j = sSrc[n];
+                        hb[q] = __ldg(A.Hbar + (int64_t)j * FF + f);
+                        xj[q] = featv(A.t, A.X, A.emb, A.types, A.N, j, f);
+                    } else {
+                        hb[q] = 0.0f;
+                        xj[q] = 0.0f;
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int n = 32 * c + q;
+                    float wb = 0.0f;
+                    if (n < ne) {
+                        const int i = sDst[n];
+                        if (i != cur) {
+                            if (cur >= 0) A.Xbar[(int64_t)cur * FF + f] += xbacc;
+                            xbacc = 0.0f;
+                            cur = i;
+                            hbi = __ldg(A.Hbar + (int64_t)i * FF + f);
+                            xi = featv(A.t, A.X, A.emb, A.types, A.N, i, f);
+                        }
+                        xbacc = fmaf(hb[q], w[q] + b2f, xbacc);
+                        wb = xj[q] * hbi + xi * hb[q];
+                    }
+                    xj[q] = wb;
+                }
+                store_tile_col<SPLIT>(Th, Tl, f, 32 * c, xj);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (f == 0) {
+                tc_fence_after();
+                issue_mma_w2<KP, SPLIT, true>(sm, tmem + COL_S);
+                mma_commit(mbar);
+            }
+            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+            // abar = sbar (.) sigma(a + b1)  (tile free again)
+#pragma unroll 1
+            for (int c = 0; c < TE / 32; ++c) {
+                float sb[32], a[32];
+                tmem_ld32(tmem + lane + COL_S + 32 * c, sb);
+                tmem_ld32(tmem + lane + COL_A + 32 * c, a);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) sb[q] *= sigmoid_t<SPLIT>(a[q] + b1f);
+                store_tile_col<SPLIT>(Th, Tl, f, 32 * c, sb);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncthreads();
+            if (f == 0) {
+                tc_fence_after();
+                issue_mma4<KP, SPLIT>(sm, tmem + COL_G);
+                mma_commit(mbar);
+            }
+            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+            // thread n = edge n: dbar = sum_k btbar[n][k] d(bt_k)/dd, force on the row owner
+            {
+                const int n = f;
+                float gsum = 0.0f;
+                const double d = sDist[n];
+                const float ratio = (float)(d / A.basis.r_cut_d);
+                const float C = 0.5f * (cospif(ratio) + 1.0f);
+                const float dC = -0.5f * (float)M_PI / A.basis.r_cut * sinpif(ratio);
+#pragma unroll 1
+                for (int c = 0; c < KP / 32; ++c) {
+                    float g[32];
+                    tmem_ld32(tmem + lane + COL_G + 32 * c, g);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) {
+                        const int k = 32 * c + q;
+                        if (n < ne && k < A.basis.K) {
+                            const float x = (float)(d - A.basis.mu[k]);
+                            const float phi = expf(-A.basis.gamma * x * x);
+                            gsum = fmaf(g[q], -2.0f * A.basis.gamma * x * phi * C + phi * dC, gsum);
+                        }
+                    }
+                }
+                sFv[3 * n] = n < ne ? -gsum * sU[3 * n] : 0.0f;
+                sFv[3 * n + 1] = n < ne ? -gsum * sU[3 * n + 1] : 0.0f;
+                sFv[3 * n + 2] = n < ne ? -gsum * sU[3 * n + 2] : 0.0f;
+            }
+            tc_fence_before();
+            __syncthreads();
+            if (f < 3) {
+                int row = sDst[0];
+                float acc = 0.0f;
+                for (int n = 0; n < ne; ++n) {
+                    if (sDst[n] != row) {
+                        A.forces[(int64_t)row * 3 + f] += acc;
+                        acc = 0.0f;
+                        row = sDst[n];
+                    }
+                    acc += sFv[3 * n + f];
+                }
+                A.forces[(int64_t)row * 3 + f] += acc;
+            }
+            __syncthreads();
+        }
+        if (ok && cur >= 0) A.Xbar[(int64_t)cur * FF + f] += xbacc;
+    }
+    teardown<KP, SPLIT>(tmem);
+}
+
+template <typename Kern>
+cudaError_t prepare(Kern k, uint32_t bytes)
+{
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int KP, bool SPLIT>
+cudaError_t launch_t(const EdgeTcArgs &a, bool backward, int G, cudaStream_t s)
+{
+    using S = TcSmem<KP, SPLIT>;
+    static_assert(S::BYTES <= 227 * 1024, "shared memory plan exceeds 227 KB");
+    cudaError_t e;
+    if (backward) {
+        if ((e = prepare(k_edge_bwd_tc<KP, SPLIT>, S::BYTES))) return e;
+        k_edge_bwd_tc<KP, SPLIT><<<G, NT, S::BYTES, s>>>(a);
+    } else {
+        if ((e = prepare(k_edge_fwd_tc<KP, SPLIT>, S::BYTES))) return e;
+        k_edge_fwd_tc<KP, SPLIT><<<G, NT, S::BYTES, s>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s)
+{
+    if (KP == 64) return split ? launch_t<64, true>(a, backward, G, s) : launch_t<64, false>(a, backward, G, s);
+    if (KP == 32) return split ? launch_t<32, true>(a, backward, G, s) : launch_t<32, false>(a, backward, G, s);
+    return cudaErrorInvalidValue;
+}
+
+// Host: one weight matrix W[rows][cols] (fp32, row-major) into the core-matrix layout used by
+// the kernels (element (r, c) at half index ((r%8)*16 + (r/8)*SBO + (c%8)*2 + (c/8)*128)/2,
+// SBO = (cols_pad/8)*128 bytes, columns cols..cols_pad-1 zero), as fp16 hi and lo = fp16(w - hi).
+void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, uint16_t *hi, uint16_t *lo)
+{
+    const size_t sbo = (size_t)(cols_pad / 8) * 128;
+    for (int r = 0; r < rows; ++r)
+        for (int c = 0; c < cols_pad; ++c) {
+            const float w = c < cols ? W[(size_t)r * cols + c] : 0.0f;
+            const __half h = __float2half_rn(w);
+            const __half l = __float2half_rn(w - __half2float(h));
+            const size_t byte = (size_t)(r % 8) * 16 + (size_t)(r / 8) * sbo + (size_t)(c % 8) * 2 + (size_t)(c / 8) * 128;
+            hi[byte / 2] = __half_as_ushort(h);
+            lo[byte / 2] = __half_as_ushort(l);
+        }
+}
+
+}  // namespace sn

@@ -42,6 +42,7 @@ enum : int {
     ERRBIT_CAPACITY = 1,
     ERRBIT_NONFINITE = 2,
     ERRBIT_DEGENERATE = 4,
+    ERRBIT_TIMEOUT = 8,
 };
 
 constexpr int NE = 32;        // edges per tile in the fp32 kernels
@@ -60,6 +61,9 @@ struct BlockW {
     const float *c1;   // [F]
     const float *U2;   // [F][F+1]
     const float *c2;   // [F]
+    // tensor-core precisions: W1 and W2 as fp16 hi / lo in the core-matrix layout of
+    // sn_ef_tc.cu (lo = fp16(w - hi), used by the split mode)
+    const void *W1h, *W1l, *W2h, *W2l;
 };
 
 struct ReadoutW {
@@ -122,6 +126,7 @@ struct EfWork {
 
 struct Model {
     int F, K, KP, T, H, n_types;
+    int precision;       // SN_PREC_*
     Basis basis;
     const float *emb;    // [n_types][F]
     BlockW blk[16];
@@ -132,6 +137,28 @@ cudaError_t launch_energy_forces(const Model &m, const sn_system &sys, const Geo
                                  const int32_t *types, const int32_t *row_ptr,
                                  const int32_t *col, EfWork &w, float *energy, float *forces,
                                  int *d_err, cudaStream_t s, Tracer *tr);
+
+// Arguments of the tensor-core edge kernels (F = 128).
+struct EdgeTcArgs {
+    const float4 *pos4;
+    const int32_t *types, *row_ptr, *col, *part;
+    const float *emb;
+    const float *X;        // [T][N][F]
+    float *H;              // [N][F]
+    const float *Hbar;     // [N][F]
+    float *Xbar;           // [N][F]
+    float *forces;         // [N][3]
+    int64_t N;
+    Geometry geo;
+    Basis basis;
+    const void *W1h, *W1l, *W2h, *W2l;
+    const float *b1, *b2;
+    int t;
+    int *d_err;
+};
+
+cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s);
+void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, uint16_t *hi, uint16_t *lo);
 
 // ---------------------------------------------------------------- integrator
 cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t n3, float c,

@@ -11,7 +11,7 @@ constexpr int RB = 256;
 
 __device__ __forceinline__ bool skip_all(const int *d_err)
 {
-    return (*((volatile const int *)d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) != 0;
+    return (*((volatile const int *)d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
 }
 
 // v += c F ; r += dt v   (c = dt/2 * kappa / m), per component
