@@ -38,6 +38,10 @@ from schnet_gnn_molecular_cell_b200 import synth  # noqa: E402
 METRIC = "energy+force evals/s and edges/s (1 B200); % of HBM/tensor roofline"
 CFG = 2
 MASS, DT, TEMP = 12.0, 2.0, 300.0
+# name -> (ABI precision, dtype string, tensor MMAs per algorithmic product)
+PRECISIONS = {"tc32": (2, "f16x2-split (fp32-accurate), f32 accumulate", 3),
+              "fp16": (1, "f16, f32 accumulate", 1),
+              "fp32": (0, "f32", 0)}
 WORKLOAD = "64 x 269-bead SAW chains, r_cut 12 A, SchNet F128 K50 T3: one velocity-Verlet step " \
            "(neighbour rebuild + energy/forces + integration)"
 
@@ -50,6 +54,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--precision", default="tc32", choices=list(PRECISIONS),
+                    help="filter-network arithmetic: tc32 = fp32-accurate fp16-split on tensor cores "
+                         "(default), fp16 = single fp16 operands (W16A16), fp32 = CUDA cores")
+    ap.add_argument("--no-variants", action="store_true", help="skip the short runs of the other precisions")
     return ap.parse_args()
 
 
@@ -163,7 +171,7 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, "fallback"
 
 
-def kernel_traffic(kernel: str, src: Path):
+def kernel_traffic(kernel: str, src: Path, precision: str = "fp32"):
     """dram bytes per launch of `kernel` from the committed ncu summary, if it was taken on
     the current source (else None)."""
     f = ROOT / "profiles" / "traffic.txt"
@@ -172,12 +180,46 @@ def kernel_traffic(kernel: str, src: Path):
     sha = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
     for line in f.read_text().splitlines():
         parts = dict(kv.split("=", 1) for kv in line.split()[1:] if "=" in kv)
-        if line.split() and line.split()[0] == kernel and parts.get("src") == sha and parts.get("workload") == "cfg2":
+        if (line.split() and line.split()[0] == kernel and parts.get("src") == sha and parts.get("workload") == "cfg2"
+                and parts.get("precision", "fp32") == precision):
             return float(parts["bytes_per_launch"])
     return None
 
 
 # ------------------------------------------------------------------------------ our arm
+def time_variant(w, v0, precision_code, steps, dev, stream, flush):
+    """Short timed run of another precision on the same workload (same protocol, no trace)."""
+    import torch
+    from schnet_gnn_molecular_cell_b200 import Context
+    s, m = w.system, w.model
+    ctx = Context(m, w.weights, stream=stream, precision=precision_code)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.from_numpy(v0.copy()).to(dev)
+    types = torch.from_numpy(w.types).to(dev)
+    rp, cl = ctx.neighbors(s, pos)
+    _, forces = ctx.energy_forces(s, pos, types, rp, cl)
+    forces = forces.clone()
+    ctx.reserve(s, int(1.5 * cl.numel()) + 4096)
+    e = torch.empty(s.n_replicas, device=dev)
+    k = torch.empty(s.n_replicas, device=dev)
+    for q in range(3):
+        flush.fill_(float(q))
+        ctx.md_step(s, pos, vel, forces, types, MASS, DT, 1, e, k)
+    ctx.sync()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for q in range(steps):
+        flush.fill_(float(q))
+        starts[q].record(stream)
+        ctx.md_step(s, pos, vel, forces, types, MASS, DT, 1, e, k)
+        ends[q].record(stream)
+    torch.cuda.synchronize()
+    ctx.sync()
+    t = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
+    ctx.close()
+    return {"value": steps / (t / 1e3), "unit": "evals/s", "ms_per_step": t / steps, "steps": steps}
+
+
 def run_ours(args):
     import torch
     rank, world, local = dist_env()
@@ -196,7 +238,8 @@ def run_ours(args):
     v0 = synth.maxwell_boltzmann(s.n_per_replica, R, MASS, TEMP, 4000 + CFG)
     stream = torch.cuda.Stream(dev)
     torch.cuda.set_stream(stream)
-    ctx = Context(m, w.weights, stream=stream)
+    prec_code, dtype, mma_per_product = PRECISIONS[args.precision]
+    ctx = Context(m, w.weights, stream=stream, precision=prec_code)
     pos = torch.from_numpy(w.pos.copy()).to(dev)
     vel = torch.from_numpy(v0.copy()).to(dev)
     types = torch.from_numpy(w.types).to(dev)
@@ -249,7 +292,8 @@ def run_ours(args):
     E_last = ctx.md_edges()
     value = world * args.steps / (t_ms / 1e3)
 
-    # dominant kernel and its roofline (algorithmic MLP flops per launch / mean launch time)
+    # dominant kernel and its roofline (algorithmic filter-network FLOPs per launch / mean
+    # launch time; the backward's forward recompute and the split's extra MMAs not counted)
     dom = max(trace, key=lambda k: trace[k][1])
     launches, dom_ms = trace[dom]
     pk, pk_kind = peaks()
@@ -257,12 +301,18 @@ def run_ours(args):
     if dom in ("edge_fwd", "edge_bwd"):
         flops = 2.0 * (m.K * m.F + m.F * m.F) * E_last
         achieved = flops / (dom_ms / launches / 1e3) / 1e12
-        fp32_peak = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        roofline = {"bound": "alu", "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s",
-                    "frac": achieved / fp32_peak,
-                    "traffic": kernel_traffic(dom, ROOT / "schnet_gnn_molecular_cell_b200" / "csrc" / "sn_ef_fp32.cu"),
-                    "kernel": dom, "peak_source": f"fp32 FMA: 148 SM x 128 lanes x 2 x {pk.get('sm_max_mhz', 1965.0):.0f} MHz ({pk_kind} sm_max_mhz)",
-                    "flops_per_launch": flops}
+        src = ROOT / "schnet_gnn_molecular_cell_b200" / "csrc" / ("sn_ef_fp32.cu" if prec_code == 0 else "sn_ef_tc.cu")
+        if prec_code == 0:
+            peak = 148 * 128 * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            bound, peak_src = "alu", (f"fp32 FMA: 148 SM x 128 lanes x 2 x {pk.get('sm_max_mhz', 1965.0):.0f} MHz "
+                                      f"({pk_kind} sm_max_mhz)")
+        else:
+            peak = pk.get("bf16_tflops_sustained", 1398.0)
+            bound, peak_src = "tensor", (f"{pk_kind} dense bf16 sustained (fp16 kind::f16 runs at the same rate); "
+                                         f"this mode issues {mma_per_product} MMA(s) per product")
+        roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": kernel_traffic(dom, src, args.precision),
+                    "kernel": dom, "peak_source": peak_src, "flops_per_launch": flops}
 
     e2e = None
     if not args.no_e2e:
@@ -296,13 +346,22 @@ def run_ours(args):
         cpu = {"value": rate, "unit": "evals/s", "cores": threads, "kind": "oracle",
                "sample": f"{steps} full velocity-Verlet step(s) of all {R} replicas in {secs:.1f} s"}
 
+    variants = None
+    if rank == 0 and world == 1 and not args.no_variants:
+        variants = {}
+        for name, (code, vdtype, _) in PRECISIONS.items():
+            if name != args.precision:
+                v = time_variant(w, v0, code, min(args.steps, 50), dev, stream, flush)
+                v["dtype"] = vdtype
+                variants[name] = v
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "evals/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
             "config": {"workload": WORKLOAD, "replicas_per_gpu": R, "beads": s.n_per_replica,
-                       "edges": E_last, "precision": "fp32 (CUDA cores)",
+                       "edges": E_last, "precision": args.precision,
                        "l2": "flushed between steps (256 MiB write, outside the timed events)",
                        "parallelism": f"{world} rank(s), independent replica batches, no collective"},
             "edges_per_s": value * E_last,
@@ -311,6 +370,7 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": sum(v[0] for v in trace.values()),
+            "precision_variants": variants,
             "clocks": clocks,
             "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0], "share": v[1] / sum(x[1] for x in trace.values())}
                         for k, v in sorted(trace.items(), key=lambda kv: -kv[1][1])},

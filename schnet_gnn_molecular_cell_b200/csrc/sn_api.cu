@@ -173,7 +173,7 @@ sn_status ensure_ef(sn_ctx *ctx, const sn_system *s)
     if ((st = grow(ctx, ctx->hbar, nf))) return st;
     if ((st = grow(ctx, ctx->xbar, nf))) return st;
     if ((st = grow(ctx, ctx->eps, sizeof(float) * N))) return st;
-    if ((st = grow(ctx, ctx->part, sizeof(int32_t) * (edge_grid(ctx) + 1)))) return st;
+    if ((st = grow(ctx, ctx->part, sizeof(int32_t) * (4 * edge_grid(ctx) + 1)))) return st;
     return SN_OK;
 }
 

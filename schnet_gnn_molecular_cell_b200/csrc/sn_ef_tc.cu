@@ -31,11 +31,14 @@ namespace sn {
 
 namespace {
 
-constexpr int TE = 128;          // edges per tile
-constexpr int NT = 128;          // threads per CTA
+constexpr int TE = 64;           // edges per tile
+constexpr int WGT = 128;         // threads per warpgroup (thread t of a group <-> TMEM lane t)
+constexpr int NWG = 2;           // warpgroups per CTA, each an independent stream of tiles
+constexpr int NT = WGT * NWG;    // threads per CTA
 constexpr int FF = 128;          // feature width supported by these kernels
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_A = 0, COL_W = 128, COL_S = 256, COL_G = 384;
+constexpr uint32_t TMEM_COLS = 256;   // per CTA: 128 columns per warpgroup
+// per-warpgroup TMEM columns: a (and later btbar) in [0, 64), w (and later sbar) in [64, 128)
+constexpr uint32_t COL_A = 0, COL_W = 64;
 constexpr float LN2F = 0.693147180559945309f;
 
 // ------------------------------------------------------------------ PTX wrappers (sm_100a)
@@ -138,32 +141,31 @@ __device__ __forceinline__ int row_of_edge(const int32_t *__restrict__ row_ptr, 
     return lo;
 }
 
-__device__ __forceinline__ uint32_t pack_h2(__half a, __half b)
-{
-    return (uint32_t)__half_as_ushort(a) | ((uint32_t)__half_as_ushort(b) << 16);
-}
 
 // 8 values -> one 16-byte fp16 run (hi) and, for SPLIT, the run of residuals (lo)
 template <bool SPLIT>
 __device__ __forceinline__ void store8(unsigned char *hi, unsigned char *lo, uint32_t off, const float *v)
 {
-    __half h[8];
+    __half2 h[4];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) h[q] = __float2half_rn(v[q]);
-    *reinterpret_cast<uint4 *>(hi + off) =
-        make_uint4(pack_h2(h[0], h[1]), pack_h2(h[2], h[3]), pack_h2(h[4], h[5]), pack_h2(h[6], h[7]));
+    for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(v[2 * q], v[2 * q + 1]);
+    *reinterpret_cast<uint4 *>(hi + off) = make_uint4(*reinterpret_cast<uint32_t *>(&h[0]), *reinterpret_cast<uint32_t *>(&h[1]),
+                                                      *reinterpret_cast<uint32_t *>(&h[2]), *reinterpret_cast<uint32_t *>(&h[3]));
     if (SPLIT) {
-        __half l[8];
+        __half2 l[4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) l[q] = __float2half_rn(v[q] - __half2float(h[q]));
-        *reinterpret_cast<uint4 *>(lo + off) =
-            make_uint4(pack_h2(l[0], l[1]), pack_h2(l[2], l[3]), pack_h2(l[4], l[5]), pack_h2(l[6], l[7]));
+        for (int q = 0; q < 4; ++q) {
+            const float2 b = __half22float2(h[q]);
+            l[q] = __floats2half2_rn(v[2 * q] - b.x, v[2 * q + 1] - b.y);
+        }
+        *reinterpret_cast<uint4 *>(lo + off) = make_uint4(*reinterpret_cast<uint32_t *>(&l[0]), *reinterpret_cast<uint32_t *>(&l[1]),
+                                                          *reinterpret_cast<uint32_t *>(&l[2]), *reinterpret_cast<uint32_t *>(&l[3]));
     }
 }
 
 // Activation tile T[n][f] (edges n contiguous in 16-byte runs): element (n, f) at
 // (n % 8) * 2 + (n / 8) * 2048 + (f % 8) * 16 + (f / 8) * 128.  Thread f stores edges
-// n0 .. n0+31 of its feature.
+// n0 .. n0+31 of its feature.  TE = 64 edges: 16 KB per fp16 copy.
 template <bool SPLIT>
 __device__ __forceinline__ void store_tile_col(unsigned char *Th, unsigned char *Tl, int f, int n0, const float (&v)[32])
 {
@@ -172,10 +174,29 @@ __device__ __forceinline__ void store_tile_col(unsigned char *Th, unsigned char 
     for (int g = 0; g < 4; ++g) store8<SPLIT>(Th, Tl, base + (uint32_t)(((n0 >> 3) + g) * 2048), v + 8 * g);
 }
 
-// Bounded wait for the MMAs committed to mbar; every thread calls it at the same point.  On
-// a time-out (never expected: nothing here waits on another agent) the error bit is set and
-// all threads return false together.
-__device__ __forceinline__ bool wait_mma(uint32_t mbar, uint32_t &phase, int *d_err)
+// Named barrier of one warpgroup (ids 1..NWG; id 0 is __syncthreads).
+__device__ __forceinline__ void wg_sync(int g)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(WGT) : "memory");
+}
+
+// Warpgroup barrier that also returns whether every thread passed a true predicate.
+__device__ __forceinline__ int wg_sync_and(int g, int pred)
+{
+    int out;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\tsetp.ne.s32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\tselp.s32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(out)
+        : "r"(pred), "r"(g + 1), "r"(WGT)
+        : "memory");
+    return out;
+}
+
+// Bounded wait for the MMAs committed to a warpgroup's mbarrier; every thread of the group
+// calls it at the same point.  On a time-out (never expected: nothing here waits on another
+// agent) the error bit is set and the whole group returns false.
+__device__ __forceinline__ bool wait_mma(int g, uint32_t mbar, uint32_t &phase, int *d_err)
 {
     const long long t0 = clock64();
     int ok = 0;
@@ -187,13 +208,13 @@ __device__ __forceinline__ bool wait_mma(uint32_t mbar, uint32_t &phase, int *d_
         if (clock64() - t0 > (1ll << 33)) break;
     }
     phase ^= 1u;
-    ok = __syncthreads_and(ok);
-    if (!ok && threadIdx.x == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
+    ok = wg_sync_and(g, ok);
+    if (!ok && (threadIdx.x % WGT) == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
     tc_fence_after();
     return ok != 0;
 }
 
-// Shared-memory plan of both kernels (bytes).
+// Shared-memory plan (bytes): weights shared by the CTA, then one region per warpgroup.
 template <int KP, bool SPLIT>
 struct TcSmem {
     static constexpr int NS = SPLIT ? 2 : 1;
@@ -201,38 +222,35 @@ struct TcSmem {
     static constexpr uint32_t W2B = FF * FF * 2;
     static constexpr uint32_t BB = TE * KP * 2;         // basis tile
     static constexpr uint32_t TB = TE * FF * 2;         // activation tile
+    static constexpr uint32_t SW1 = (KP / 8) * 128;     // 8-row group stride of W1 and of the basis tile
     static constexpr uint32_t W1 = 0;
     static constexpr uint32_t W2 = W1 + NS * W1B;
-    static constexpr uint32_t B = W2 + NS * W2B;
+    static constexpr uint32_t GROUPS = W2 + NS * W2B;
+    // offsets inside a warpgroup region
+    static constexpr uint32_t B = 0;
     static constexpr uint32_t T = B + NS * BB;
-    static constexpr uint32_t META = T + NS * TB;       // src, dst (int), d (double), u[3], fv[3] (float)
-    static constexpr uint32_t SRC = META;
-    static constexpr uint32_t DST = SRC + 4 * TE;
-    static constexpr uint32_t DIST = DST + 4 * TE;
-    static constexpr uint32_t UVEC = DIST + 8 * TE;
-    static constexpr uint32_t FV = UVEC + 12 * TE;
-    static constexpr uint32_t MBAR = FV + 12 * TE;
-    static constexpr uint32_t HOLD = MBAR + 8;
+    static constexpr uint32_t SRC = T + NS * TB;        // int[TE]
+    static constexpr uint32_t DST = SRC + 4 * TE;       // int[TE]
+    static constexpr uint32_t DIST = DST + 4 * TE;      // double[TE]
+    static constexpr uint32_t UVEC = DIST + 8 * TE;     // float[TE][3]
+    static constexpr uint32_t FV = UVEC + 12 * TE;      // float[TE][3]
+    static constexpr uint32_t MBAR = FV + 12 * TE;      // uint64
+    static constexpr uint32_t REGION = (MBAR + 8 + 127) / 128 * 128;
+    static constexpr uint32_t HOLD = GROUPS + NWG * REGION;
     static constexpr uint32_t USED = HOLD + 16;
-    // at least 116 KB so that no two CTAs share an SM (each allocates all 512 TMEM columns)
+    // at least 116 KB so that no two CTAs share an SM
     static constexpr uint32_t BYTES = USED > 116 * 1024 ? USED : 116 * 1024;
-    static constexpr uint32_t SW1 = (KP / 8) * 128;     // 8-row group stride of W1 and of the basis tile
 };
 
 }  // namespace
 
 namespace {
 
-template <bool ACCURATE>
-__device__ __forceinline__ float ssp_t(float x)
-{
-    return fmaxf(x, 0.0f) + log1pf(ACCURATE ? expf(-fabsf(x)) : __expf(-fabsf(x))) - LN2F;
-}
-template <bool ACCURATE>
-__device__ __forceinline__ float sigmoid_t(float x)
-{
-    return ACCURATE ? 1.0f / (1.0f + expf(-x)) : __fdividef(1.0f, 1.0f + __expf(-x));
-}
+// Activations with the hardware exp2/log2 units (__expf, __logf): ssp(x) = max(x, 0) +
+// ln(1 + e^-|x|) - ln 2 and sigma(x) = 1 / (1 + e^-x).  Absolute error ~3e-7, below the
+// 2^-22 resolution of the split fp16 operands they feed.
+__device__ __forceinline__ float ssp_fast(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))) - LN2F; }
+__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
 __device__ __forceinline__ void copy_to_smem(unsigned char *dst, const void *src, uint32_t bytes)
 {
@@ -241,18 +259,20 @@ __device__ __forceinline__ void copy_to_smem(unsigned char *dst, const void *src
     for (uint32_t q = threadIdx.x; q < bytes / 16; q += NT) d[q] = __ldg(s + q);
 }
 
-// Edge metadata and the basis row of edge n = threadIdx.x: u = r_i - r_j and d in double
-// (minimum image on periodic axes), unit vector, and bt_k = exp(-gamma (d - mu_k)^2) C(d) as
-// fp16 (hi/lo) in the basis tile; zero for k >= K and for padding edges n >= ne.
+// Edge metadata and basis rows of one tile, by the 128 threads of a warpgroup: thread t
+// handles edge n = t % 64 and half of its K_P Gaussians.  u = r_i - r_j and d in double
+// (minimum image on periodic axes); bt_k = exp(-gamma (d - mu_k)^2) C(d) as fp16 (hi/lo);
+// zero for k >= K and for padding edges n >= ne.
 template <int KP, bool SPLIT>
-__device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char *sm, int i0, int i1, int ts, int ne)
+__device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char *R, int t, int i0, int i1, int ts,
+                                              int ne)
 {
     using S = TcSmem<KP, SPLIT>;
-    const int n = threadIdx.x;
-    int *sSrc = reinterpret_cast<int *>(sm + S::SRC);
-    int *sDst = reinterpret_cast<int *>(sm + S::DST);
-    double *sDist = reinterpret_cast<double *>(sm + S::DIST);
-    float *sU = reinterpret_cast<float *>(sm + S::UVEC);
+    const int n = t & (TE - 1), half = t / TE;
+    int *sSrc = reinterpret_cast<int *>(R + S::SRC);
+    int *sDst = reinterpret_cast<int *>(R + S::DST);
+    double *sDist = reinterpret_cast<double *>(R + S::DIST);
+    float *sU = reinterpret_cast<float *>(R + S::UVEC);
     double d = 0.0;
     if (n < ne) {
         const int e = ts + n;
@@ -264,23 +284,26 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
         if (A.geo.periodic[1]) dy -= (double)A.geo.box[1] * rint(dy / (double)A.geo.box[1]);
         if (A.geo.periodic[2]) dz -= (double)A.geo.box[2] * rint(dz / (double)A.geo.box[2]);
         d = sqrt(dx * dx + dy * dy + dz * dz);
-        sSrc[n] = j;
-        sDst[n] = i;
-        sDist[n] = d;
-        sU[3 * n] = (float)(dx / d);
-        sU[3 * n + 1] = (float)(dy / d);
-        sU[3 * n + 2] = (float)(dz / d);
-    } else {
+        if (half == 0) {
+            sSrc[n] = j;
+            sDst[n] = i;
+            sDist[n] = d;
+            sU[3 * n] = (float)(dx / d);
+            sU[3 * n + 1] = (float)(dy / d);
+            sU[3 * n + 2] = (float)(dz / d);
+        }
+    } else if (half == 0) {
         sSrc[n] = -1;
         sDst[n] = -1;
         sDist[n] = 0.0;
     }
     const float C = 0.5f * (cospif((float)(d / A.basis.r_cut_d)) + 1.0f);
-    unsigned char *Bh = sm + S::B;
+    unsigned char *Bh = R + S::B;
     unsigned char *Bl = Bh + S::BB;
     const uint32_t row = (uint32_t)((n & 7) * 16 + (n >> 3) * S::SW1);
 #pragma unroll
-    for (int q = 0; q < KP / 8; ++q) {
+    for (int qq = 0; qq < KP / 16; ++qq) {
+        const int q = half * (KP / 16) + qq;
         float v[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -296,14 +319,14 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
     }
 }
 
-// D_A[f][n] = sum_k W1[f][k] bt[n][k]
+// D_A[f][n] = sum_k W1[f][k] bt[n][k]                          (M = 128, N = TE)
 template <int KP, bool SPLIT>
-__device__ __forceinline__ void issue_mma1(unsigned char *sm, uint32_t d)
+__device__ __forceinline__ void issue_mma1(unsigned char *sm, unsigned char *R, uint32_t d)
 {
     using S = TcSmem<KP, SPLIT>;
     constexpr uint32_t ID = idesc_f16(128, TE, 0, 0);
     const uint32_t wh = smem_u32(sm + S::W1), wl = wh + S::W1B;
-    const uint32_t bh = smem_u32(sm + S::B), bl = bh + S::BB;
+    const uint32_t bh = smem_u32(R + S::B), bl = bh + S::BB;
 #pragma unroll
     for (int j = 0; j < KP / 16; ++j) {
         const uint32_t o = (uint32_t)j * 256;
@@ -318,12 +341,12 @@ __device__ __forceinline__ void issue_mma1(unsigned char *sm, uint32_t d)
 // TRANS = false: D[o][n] = sum_i W2[o][i] T[n][i]   (forward filter layer 2)
 // TRANS = true : D[i][n] = sum_o W2[o][i] T[n][o]   (backward through layer 2)
 template <int KP, bool SPLIT, bool TRANS>
-__device__ __forceinline__ void issue_mma_w2(unsigned char *sm, uint32_t d)
+__device__ __forceinline__ void issue_mma_w2(unsigned char *sm, unsigned char *R, uint32_t d)
 {
     using S = TcSmem<KP, SPLIT>;
     constexpr uint32_t ID = idesc_f16(128, TE, TRANS ? 1 : 0, 1);
     const uint32_t wh = smem_u32(sm + S::W2), wl = wh + S::W2B;
-    const uint32_t th = smem_u32(sm + S::T), tl = th + S::TB;
+    const uint32_t th = smem_u32(R + S::T), tl = th + S::TB;
     const uint32_t a_lbo = TRANS ? 2048 : 128, a_sbo = TRANS ? 128 : 2048, a_step = TRANS ? 4096 : 256;
 #pragma unroll
     for (int j = 0; j < FF / 16; ++j) {
@@ -336,14 +359,15 @@ __device__ __forceinline__ void issue_mma_w2(unsigned char *sm, uint32_t d)
     }
 }
 
-// D_G[n][k] = sum_f abar[n][f] W1[f][k]   (edges on M)
+// D_G[n][k] = sum_f abar[n][f] W1[f][k]   (edges on M: M = TE = 64; row n of D sits in TMEM
+// lane (n % 16) + 32 (n / 16))
 template <int KP, bool SPLIT>
-__device__ __forceinline__ void issue_mma4(unsigned char *sm, uint32_t d)
+__device__ __forceinline__ void issue_mma4(unsigned char *sm, unsigned char *R, uint32_t d)
 {
     using S = TcSmem<KP, SPLIT>;
-    constexpr uint32_t ID = idesc_f16(128, KP, 1, 1);
+    constexpr uint32_t ID = idesc_f16(TE, KP, 1, 1);
     const uint32_t wh = smem_u32(sm + S::W1), wl = wh + S::W1B;
-    const uint32_t th = smem_u32(sm + S::T), tl = th + S::TB;
+    const uint32_t th = smem_u32(R + S::T), tl = th + S::TB;
 #pragma unroll
     for (int j = 0; j < FF / 16; ++j) {
         const uint32_t oa = (uint32_t)j * 256, ob = (uint32_t)j * 2 * S::SW1;
@@ -355,7 +379,7 @@ __device__ __forceinline__ void issue_mma4(unsigned char *sm, uint32_t d)
     }
 }
 
-// Common kernel set-up: weights to shared memory, mbarrier, TMEM allocation.
+// Kernel set-up: weights to shared memory, one mbarrier per warpgroup, TMEM for the CTA.
 template <int KP, bool SPLIT>
 __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm, int &skip)
 {
@@ -368,7 +392,7 @@ __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm
         copy_to_smem(sm + S::W2 + S::W2B, A.W2l, S::W2B);
     }
     if (threadIdx.x == 0) {
-        mbar_init(smem_u32(sm + S::MBAR), 1);
+        for (int g = 0; g < NWG; ++g) mbar_init(smem_u32(sm + S::GROUPS + g * S::REGION + S::MBAR), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     }
@@ -380,7 +404,6 @@ __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm
     return *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
 }
 
-template <int KP, bool SPLIT>
 __device__ __forceinline__ void teardown(uint32_t tmem)
 {
     tc_fence_before();
@@ -389,63 +412,88 @@ __device__ __forceinline__ void teardown(uint32_t tmem)
     if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+// Per-warpgroup context: group g, thread t in group (= TMEM lane = feature), its shared region,
+// mbarrier, TMEM columns and row range.
+struct Group {
+    int g, t;
+    unsigned char *R;
+    uint32_t mbar, tm, lane;
+    int i0, i1;
+};
+
+template <int KP, bool SPLIT>
+__device__ __forceinline__ Group make_group(const EdgeTcArgs &A, unsigned char *sm, uint32_t tmem0)
+{
+    using S = TcSmem<KP, SPLIT>;
+    Group G;
+    G.g = threadIdx.x / WGT;
+    G.t = threadIdx.x % WGT;
+    G.R = sm + S::GROUPS + G.g * S::REGION;
+    G.mbar = smem_u32(G.R + S::MBAR);
+    G.tm = tmem0 + (uint32_t)G.g * 128;
+    G.lane = (uint32_t)((G.t >> 5) * 32) << 16;
+    const int p = blockIdx.x * NWG + G.g;
+    G.i0 = A.part[p];
+    G.i1 = A.part[p + 1];
+    return G;
+}
+
+// Make this group's shared-memory writes visible to the tensor core, then let thread 0 of the
+// group issue the MMAs of `issue` and commit them to the group's mbarrier; all threads wait.
+template <typename Issue>
+__device__ __forceinline__ bool mma_step(const Group &G, uint32_t &phase, int *d_err, Issue issue)
+{
+    fence_async_smem();
+    tc_fence_before();
+    wg_sync(G.g);
+    if (G.t == 0) {
+        tc_fence_after();
+        issue();
+        mma_commit(G.mbar);
+    }
+    return wait_mma(G.g, G.mbar, phase, d_err);
+}
+
 template <int KP, bool SPLIT>
 __global__ void __launch_bounds__(NT, 1) k_edge_fwd_tc(EdgeTcArgs A)
 {
     using S = TcSmem<KP, SPLIT>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
-    const int f = threadIdx.x, warp = f >> 5;
-    const uint32_t tmem = setup<KP, SPLIT>(A, sm, skip);
-    const uint32_t mbar = smem_u32(sm + S::MBAR);
-    const uint32_t lane = (uint32_t)(warp * 32) << 16;
-    const int i0 = A.part[blockIdx.x], i1 = A.part[blockIdx.x + 1];
-    if (!skip && i0 < i1) {
-        const int e0 = A.row_ptr[i0], e1 = A.row_ptr[i1];
+    const uint32_t tmem0 = setup<KP, SPLIT>(A, sm, skip);
+    const Group G = make_group<KP, SPLIT>(A, sm, tmem0);
+    const int f = G.t;
+    if (!skip && G.i0 < G.i1) {
+        const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
         const float b1f = A.b1[f], b2f = A.b2[f];
-        const int *sSrc = reinterpret_cast<const int *>(sm + S::SRC);
-        const int *sDst = reinterpret_cast<const int *>(sm + S::DST);
-        unsigned char *Th = sm + S::T, *Tl = Th + S::TB;
+        const int *sSrc = reinterpret_cast<const int *>(G.R + S::SRC);
+        const int *sDst = reinterpret_cast<const int *>(G.R + S::DST);
+        unsigned char *Th = G.R + S::T, *Tl = Th + S::TB;
         uint32_t phase = 0;
-        int cur = i0;
+        int cur = G.i0;
         float hacc = 0.0f;
         bool ok = true;
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT>(A, sm, i0, i1, ts, ne);
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (f == 0) {
-                tc_fence_after();
-                issue_mma1<KP, SPLIT>(sm, tmem + COL_A);
-                mma_commit(mbar);
-            }
-            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+            tile_prologue<KP, SPLIT>(A, G.R, f, G.i0, G.i1, ts, ne);
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
             // s = ssp(a + b1) into the activation tile
 #pragma unroll 1
             for (int c = 0; c < TE / 32; ++c) {
                 float v[32];
-                tmem_ld32(tmem + lane + COL_A + 32 * c, v);
+                tmem_ld32(G.tm + G.lane + COL_A + 32 * c, v);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] = ssp_t<SPLIT>(v[q] + b1f);
+                for (int q = 0; q < 32; ++q) v[q] = ssp_fast(v[q] + b1f);
                 store_tile_col<SPLIT>(Th, Tl, f, 32 * c, v);
             }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (f == 0) {
-                tc_fence_after();
-                issue_mma_w2<KP, SPLIT, false>(sm, tmem + COL_W);
-                mma_commit(mbar);
-            }
-            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
+                break;
             // h_i += x_src (.) (w + b2), segment sums per destination row
 #pragma unroll 1
             for (int c = 0; c < TE / 32; ++c) {
                 if (32 * c >= ne) break;
                 float v[32], xs[32];
-                tmem_ld32(tmem + lane + COL_W + 32 * c, v);
+                tmem_ld32(G.tm + G.lane + COL_W + 32 * c, v);
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const int n = 32 * c + q;
@@ -467,185 +515,154 @@ __global__ void __launch_bounds__(NT, 1) k_edge_fwd_tc(EdgeTcArgs A)
                 }
             }
             tc_fence_before();
-            __syncthreads();
+            wg_sync(G.g);
         }
         if (ok) {
             A.H[(int64_t)cur * FF + f] = hacc;
-            for (int r = cur + 1; r < i1; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
+            for (int r = cur + 1; r < G.i1; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
         }
     }
-    teardown<KP, SPLIT>(tmem);
+    teardown(tmem0);
 }
 
-// Backward of one interaction block over the CTA's rows (see sn_ef_fp32.cu for the algebra):
+// Backward of one interaction block over the group's rows (see sn_ef_fp32.cu for the algebra):
 // recompute a = W1 bt + b1 and w = W2 ssp(a) + b2; xbar_i += sum_j hbar_j (.) w_ij;
 // wbar = x_j (.) hbar_i + x_i (.) hbar_j; sbar = W2^T wbar; abar = sbar (.) sigma(a);
-// btbar = W1^T abar (edges on M, one TMEM lane per edge); dbar = btbar . d(bt)/dd;
-// F_i -= dbar * u_ij / d_ij, accumulated by the row's owner only.
+// btbar = W1^T abar (edges on M); dbar = btbar . d(bt)/dd; F_i -= dbar * u_ij / d_ij by the
+// row's owner only.  TMEM columns are reused: sbar overwrites w, btbar overwrites a.
 template <int KP, bool SPLIT>
 __global__ void __launch_bounds__(NT, 1) k_edge_bwd_tc(EdgeTcArgs A)
 {
     using S = TcSmem<KP, SPLIT>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
-    const int f = threadIdx.x, warp = f >> 5;
-    const uint32_t tmem = setup<KP, SPLIT>(A, sm, skip);
-    const uint32_t mbar = smem_u32(sm + S::MBAR);
-    const uint32_t lane = (uint32_t)(warp * 32) << 16;
-    const int i0 = A.part[blockIdx.x], i1 = A.part[blockIdx.x + 1];
-    if (!skip && i0 < i1) {
-        const int e0 = A.row_ptr[i0], e1 = A.row_ptr[i1];
+    const uint32_t tmem0 = setup<KP, SPLIT>(A, sm, skip);
+    const Group G = make_group<KP, SPLIT>(A, sm, tmem0);
+    const int f = G.t;
+    if (!skip && G.i0 < G.i1) {
+        const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
         const float b1f = A.b1[f], b2f = A.b2[f];
-        const int *sSrc = reinterpret_cast<const int *>(sm + S::SRC);
-        const int *sDst = reinterpret_cast<const int *>(sm + S::DST);
-        const double *sDist = reinterpret_cast<const double *>(sm + S::DIST);
-        const float *sU = reinterpret_cast<const float *>(sm + S::UVEC);
-        float *sFv = reinterpret_cast<float *>(sm + S::FV);
-        unsigned char *Th = sm + S::T, *Tl = Th + S::TB;
+        const int *sSrc = reinterpret_cast<const int *>(G.R + S::SRC);
+        const int *sDst = reinterpret_cast<const int *>(G.R + S::DST);
+        const double *sDist = reinterpret_cast<const double *>(G.R + S::DIST);
+        const float *sU = reinterpret_cast<const float *>(G.R + S::UVEC);
+        float *sFv = reinterpret_cast<float *>(G.R + S::FV);
+        unsigned char *Th = G.R + S::T, *Tl = Th + S::TB;
         uint32_t phase = 0;
         int cur = -1;
-        float xbacc = 0.0f, hbi = 0.0f, xi = 0.0f;
+        float xbacc = 0.0f, xbold = 0.0f;
         bool ok = true;
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT>(A, sm, i0, i1, ts, ne);
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (f == 0) {
-                tc_fence_after();
-                issue_mma1<KP, SPLIT>(sm, tmem + COL_A);
-                mma_commit(mbar);
-            }
-            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
+            tile_prologue<KP, SPLIT>(A, G.R, f, G.i0, G.i1, ts, ne);
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
 #pragma unroll 1
             for (int c = 0; c < TE / 32; ++c) {
                 float v[32];
-                tmem_ld32(tmem + lane + COL_A + 32 * c, v);
+                tmem_ld32(G.tm + G.lane + COL_A + 32 * c, v);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] = ssp_t<SPLIT>(v[q] + b1f);
+                for (int q = 0; q < 32; ++q) v[q] = ssp_fast(v[q] + b1f);
                 store_tile_col<SPLIT>(Th, Tl, f, 32 * c, v);
             }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (f == 0) {
-                tc_fence_after();
-                issue_mma_w2<KP, SPLIT, false>(sm, tmem + COL_W);
-                mma_commit(mbar);
-            }
-            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
-            // xbar and wbar (the activation tile is free: the MMA that read s has completed)
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
+                break;
+            // xbar and wbar; source and destination features of a chunk are loaded up front
 #pragma unroll 1
             for (int c = 0; c < TE / 32; ++c) {
-                float w[32], hb[32], xj[32];
-                tmem_ld32(tmem + lane + COL_W + 32 * c, w);
+                float w[32], hb[32], xj[32], hi_[32], xi_[32];
+                tmem_ld32(G.tm + G.lane + COL_W + 32 * c, w);
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const int n = 32 * c + q;
                     if (n < ne) {
-                        const int j = sSrc[n];
+                        const int j = sSrc[n], i = sDst[n];
                         hb[q] = __ldg(A.Hbar + (int64_t)j * FF + f);
                         xj[q] = featv(A.t, A.X, A.emb, A.types, A.N, j, f);
+                        hi_[q] = __ldg(A.Hbar + (int64_t)i * FF + f);
+                        xi_[q] = featv(A.t, A.X, A.emb, A.types, A.N, i, f);
                     } else {
-                        hb[q] = 0.0f;
-                        xj[q] = 0.0f;
+                        hb[q] = xj[q] = hi_[q] = xi_[q] = 0.0f;
                     }
                 }
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const int n = 32 * c + q;
-                    float wb = 0.0f;
                     if (n < ne) {
                         const int i = sDst[n];
                         if (i != cur) {
-                            if (cur >= 0) A.Xbar[(int64_t)cur * FF + f] += xbacc;
+                            if (cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
                             xbacc = 0.0f;
                             cur = i;
-                            hbi = __ldg(A.Hbar + (int64_t)i * FF + f);
-                            xi = featv(A.t, A.X, A.emb, A.types, A.N, i, f);
+                            xbold = A.Xbar[(int64_t)i * FF + f];   // consumed at this row's flush
                         }
                         xbacc = fmaf(hb[q], w[q] + b2f, xbacc);
-                        wb = xj[q] * hbi + xi * hb[q];
                     }
-                    xj[q] = wb;
+                    xj[q] = n < ne ? xj[q] * hi_[q] + xi_[q] * hb[q] : 0.0f;
                 }
                 store_tile_col<SPLIT>(Th, Tl, f, 32 * c, xj);
             }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (f == 0) {
-                tc_fence_after();
-                issue_mma_w2<KP, SPLIT, true>(sm, tmem + COL_S);
-                mma_commit(mbar);
-            }
-            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
-            // abar = sbar (.) sigma(a + b1)  (tile free again)
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, true>(sm, G.R, G.tm + COL_W); })))
+                break;
+            // abar = sbar (.) sigma(a + b1)
 #pragma unroll 1
             for (int c = 0; c < TE / 32; ++c) {
                 float sb[32], a[32];
-                tmem_ld32(tmem + lane + COL_S + 32 * c, sb);
-                tmem_ld32(tmem + lane + COL_A + 32 * c, a);
+                tmem_ld32(G.tm + G.lane + COL_W + 32 * c, sb);
+                tmem_ld32(G.tm + G.lane + COL_A + 32 * c, a);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) sb[q] *= sigmoid_t<SPLIT>(a[q] + b1f);
+                for (int q = 0; q < 32; ++q) sb[q] *= sigmoid_fast(a[q] + b1f);
                 store_tile_col<SPLIT>(Th, Tl, f, 32 * c, sb);
             }
-            fence_async_smem();
-            tc_fence_before();
-            __syncthreads();
-            if (f == 0) {
-                tc_fence_after();
-                issue_mma4<KP, SPLIT>(sm, tmem + COL_G);
-                mma_commit(mbar);
-            }
-            if (!(ok = wait_mma(mbar, phase, A.d_err))) break;
-            // thread n = edge n: dbar = sum_k btbar[n][k] d(bt_k)/dd, force on the row owner
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma4<KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
+            // lanes 0-15 of each warp quadrant: edge n = 16 * quadrant + lane, dbar and force
             {
-                const int n = f;
+                const int l = f & 31, n = (f >> 5) * 16 + l;
                 float gsum = 0.0f;
-                const double d = sDist[n];
+                const bool mine = l < 16 && n < ne;
+                const double d = mine ? sDist[n] : 0.0;
                 const float ratio = (float)(d / A.basis.r_cut_d);
                 const float C = 0.5f * (cospif(ratio) + 1.0f);
                 const float dC = -0.5f * (float)M_PI / A.basis.r_cut * sinpif(ratio);
 #pragma unroll 1
                 for (int c = 0; c < KP / 32; ++c) {
-                    float g[32];
-                    tmem_ld32(tmem + lane + COL_G + 32 * c, g);
+                    float gg[32];
+                    tmem_ld32(G.tm + G.lane + COL_A + 32 * c, gg);
 #pragma unroll
                     for (int q = 0; q < 32; ++q) {
                         const int k = 32 * c + q;
-                        if (n < ne && k < A.basis.K) {
+                        if (mine && k < A.basis.K) {
                             const float x = (float)(d - A.basis.mu[k]);
                             const float phi = expf(-A.basis.gamma * x * x);
-                            gsum = fmaf(g[q], -2.0f * A.basis.gamma * x * phi * C + phi * dC, gsum);
+                            gsum = fmaf(gg[q], -2.0f * A.basis.gamma * x * phi * C + phi * dC, gsum);
                         }
                     }
                 }
-                sFv[3 * n] = n < ne ? -gsum * sU[3 * n] : 0.0f;
-                sFv[3 * n + 1] = n < ne ? -gsum * sU[3 * n + 1] : 0.0f;
-                sFv[3 * n + 2] = n < ne ? -gsum * sU[3 * n + 2] : 0.0f;
+                if (l < 16) {
+                    sFv[3 * n] = mine ? -gsum * sU[3 * n] : 0.0f;
+                    sFv[3 * n + 1] = mine ? -gsum * sU[3 * n + 1] : 0.0f;
+                    sFv[3 * n + 2] = mine ? -gsum * sU[3 * n + 2] : 0.0f;
+                }
             }
             tc_fence_before();
-            __syncthreads();
-            if (f < 3) {
-                int row = sDst[0];
-                float acc = 0.0f;
-                for (int n = 0; n < ne; ++n) {
-                    if (sDst[n] != row) {
-                        A.forces[(int64_t)row * 3 + f] += acc;
-                        acc = 0.0f;
-                        row = sDst[n];
-                    }
-                    acc += sFv[3 * n + f];
+            wg_sync(G.g);
+            // one thread per row segment of the tile sums its edges' forces in edge order
+            if (f < ne && (f == 0 || sDst[f] != sDst[f - 1])) {
+                const int row = sDst[f];
+                float fx = 0.0f, fy = 0.0f, fz = 0.0f;
+                for (int n = f; n < ne && sDst[n] == row; ++n) {
+                    fx += sFv[3 * n];
+                    fy += sFv[3 * n + 1];
+                    fz += sFv[3 * n + 2];
                 }
-                A.forces[(int64_t)row * 3 + f] += acc;
+                A.forces[(int64_t)row * 3] += fx;
+                A.forces[(int64_t)row * 3 + 1] += fy;
+                A.forces[(int64_t)row * 3 + 2] += fz;
             }
-            __syncthreads();
+            wg_sync(G.g);
         }
-        if (ok && cur >= 0) A.Xbar[(int64_t)cur * FF + f] += xbacc;
+        if (ok && cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
     }
-    teardown<KP, SPLIT>(tmem);
+    teardown(tmem0);
 }
 
 template <typename Kern>
@@ -672,6 +689,9 @@ cudaError_t launch_t(const EdgeTcArgs &a, bool backward, int G, cudaStream_t s)
 
 }  // namespace
 
+int tc_groups_per_cta() { return NWG; }
+
+// G CTAs, each running NWG independent row ranges: a.part must hold G * NWG + 1 entries.
 cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s)
 {
     if (KP == 64) return split ? launch_t<64, true>(a, backward, G, s) : launch_t<64, false>(a, backward, G, s);

@@ -120,7 +120,7 @@ struct EfWork {
     float *hbar;         // [N][F]      dE/dh of the current block
     float *xbar;         // [N][F]      dE/dx of the current block (in place)
     float *eps;          // [N]         per-atom energies
-    int32_t *part;       // [G + 1]     rows owned by each CTA of the edge kernels
+    int32_t *part;       // [4 G + 1]   rows owned by each CTA (fp32) / warpgroup (tensor cores)
     int G;
 };
 
@@ -158,6 +158,7 @@ struct EdgeTcArgs {
 };
 
 cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s);
+int tc_groups_per_cta();   // independent row ranges per CTA of the tensor-core edge kernels
 void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, uint16_t *hi, uint16_t *lo);
 
 // ---------------------------------------------------------------- integrator
