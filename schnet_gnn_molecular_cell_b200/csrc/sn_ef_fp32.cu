@@ -617,7 +617,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
     if ((e = set_smem(k_node_bwd<F>, nb_bytes))) return e;
 
     trace_begin(tr, KK_PARTITION, s);
-    const int parts = m.precision == SN_PREC_FP32 ? w.G : w.G * tc_groups_per_cta();
+    const int parts = m.precision == SN_PREC_FP32 ? w.G : w.G * tc_groups_per_cta(m.precision == SN_PREC_TC32);
     k_partition<<<(parts + 1 + 127) / 128, 128, 0, s>>>(row_ptr, N, parts, w.part);
     trace_end(tr, s);
 

@@ -33,10 +33,8 @@ namespace {
 
 constexpr int TE = 64;           // edges per tile
 constexpr int WGT = 128;         // threads per warpgroup (thread t of a group <-> TMEM lane t)
-constexpr int NWG = 2;           // warpgroups per CTA, each an independent stream of tiles
-constexpr int NT = WGT * NWG;    // threads per CTA
 constexpr int FF = 128;          // feature width supported by these kernels
-constexpr uint32_t TMEM_COLS = 256;   // per CTA: 128 columns per warpgroup
+// TMEM: 128 columns per warpgroup (128 * NW per CTA)
 // per-warpgroup TMEM columns: a (and later btbar) in [0, 64), w (and later sbar) in [64, 128)
 constexpr uint32_t COL_A = 0, COL_W = 64;
 constexpr float LN2F = 0.693147180559945309f;
@@ -108,6 +106,28 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// This lane's 16 consecutive 32-bit TMEM columns starting at taddr.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+template <int CH>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[CH])
+{
+    if constexpr (CH == 32) tmem_ld32(taddr, v);
+    else tmem_ld16(taddr, v);
+}
+
 // Shared-memory matrix descriptor, no swizzle (layout type 0), version 1.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
@@ -123,12 +143,6 @@ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major)
 }
 
 // ------------------------------------------------------------------ helpers
-__device__ __forceinline__ float featv(int t, const float *__restrict__ X, const float *__restrict__ emb,
-                                       const int32_t *__restrict__ types, int64_t N, int j, int f)
-{
-    if (t == 0) return __ldg(emb + (int64_t)__ldg(types + j) * FF + f);
-    return __ldg(X + ((int64_t)(t - 1) * N + j) * FF + f);
-}
 
 __device__ __forceinline__ int row_of_edge(const int32_t *__restrict__ row_ptr, int i0, int i1, int e)
 {
@@ -166,15 +180,15 @@ __device__ __forceinline__ void store8(unsigned char *hi, unsigned char *lo, uin
 // Activation tile T[n][f] (edges n contiguous in 16-byte runs): element (n, f) at
 // (n % 8) * 2 + (n / 8) * 2048 + (f % 8) * 16 + (f / 8) * 128.  Thread f stores edges
 // n0 .. n0+31 of its feature.  TE = 64 edges: 16 KB per fp16 copy.
-template <bool SPLIT>
-__device__ __forceinline__ void store_tile_col(unsigned char *Th, unsigned char *Tl, int f, int n0, const float (&v)[32])
+template <bool SPLIT, int CH>
+__device__ __forceinline__ void store_tile_col(unsigned char *Th, unsigned char *Tl, int f, int n0, const float (&v)[CH])
 {
     const uint32_t base = (uint32_t)((f & 7) * 16 + (f >> 3) * 128);
 #pragma unroll
-    for (int g = 0; g < 4; ++g) store8<SPLIT>(Th, Tl, base + (uint32_t)(((n0 >> 3) + g) * 2048), v + 8 * g);
+    for (int g = 0; g < CH / 8; ++g) store8<SPLIT>(Th, Tl, base + (uint32_t)(((n0 >> 3) + g) * 2048), v + 8 * g);
 }
 
-// Named barrier of one warpgroup (ids 1..NWG; id 0 is __syncthreads).
+// Named barrier of one warpgroup (ids 1..4; id 0 is __syncthreads).
 __device__ __forceinline__ void wg_sync(int g)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(WGT) : "memory");
@@ -215,7 +229,7 @@ __device__ __forceinline__ bool wait_mma(int g, uint32_t mbar, uint32_t &phase, 
 }
 
 // Shared-memory plan (bytes): weights shared by the CTA, then one region per warpgroup.
-template <int KP, bool SPLIT>
+template <int KP, bool SPLIT, int NW>
 struct TcSmem {
     static constexpr int NS = SPLIT ? 2 : 1;
     static constexpr uint32_t W1B = FF * KP * 2;        // one fp16 copy of W1
@@ -229,14 +243,17 @@ struct TcSmem {
     // offsets inside a warpgroup region
     static constexpr uint32_t B = 0;
     static constexpr uint32_t T = B + NS * BB;
-    static constexpr uint32_t SRC = T + NS * TB;        // int[TE]
-    static constexpr uint32_t DST = SRC + 4 * TE;       // int[TE]
-    static constexpr uint32_t DIST = DST + 4 * TE;      // double[TE]
-    static constexpr uint32_t UVEC = DIST + 8 * TE;     // float[TE][3]
+    static constexpr uint32_t PX = T + NS * TB;         // const float *[TE]: x row of the source
+    static constexpr uint32_t PH = PX + 8 * TE;         //                    hbar row of the source
+    static constexpr uint32_t PXI = PH + 8 * TE;        //                    x row of the destination
+    static constexpr uint32_t PHI = PXI + 8 * TE;       //                    hbar row of the destination
+    static constexpr uint32_t DIST = PHI + 8 * TE;      // double[TE]
+    static constexpr uint32_t DST = DIST + 8 * TE;      // int[TE]
+    static constexpr uint32_t UVEC = DST + 4 * TE;      // float[TE][3]
     static constexpr uint32_t FV = UVEC + 12 * TE;      // float[TE][3]
     static constexpr uint32_t MBAR = FV + 12 * TE;      // uint64
     static constexpr uint32_t REGION = (MBAR + 8 + 127) / 128 * 128;
-    static constexpr uint32_t HOLD = GROUPS + NWG * REGION;
+    static constexpr uint32_t HOLD = GROUPS + NW * REGION;
     static constexpr uint32_t USED = HOLD + 16;
     // at least 116 KB so that no two CTAs share an SM
     static constexpr uint32_t BYTES = USED > 116 * 1024 ? USED : 116 * 1024;
@@ -252,24 +269,36 @@ namespace {
 __device__ __forceinline__ float ssp_fast(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))) - LN2F; }
 __device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
+template <int NW>
 __device__ __forceinline__ void copy_to_smem(unsigned char *dst, const void *src, uint32_t bytes)
 {
     const uint4 *s = reinterpret_cast<const uint4 *>(src);
     uint4 *d = reinterpret_cast<uint4 *>(dst);
-    for (uint32_t q = threadIdx.x; q < bytes / 16; q += NT) d[q] = __ldg(s + q);
+    for (uint32_t q = threadIdx.x; q < bytes / 16; q += WGT * NW) d[q] = __ldg(s + q);
+}
+
+__device__ __forceinline__ const float *feat_row(const EdgeTcArgs &A, int j)
+{
+    // x^0 is the embedding of the type; x^t (t >= 1) lives in X[t-1]
+    if (A.t == 0) return A.emb + (int64_t)__ldg(A.types + j) * FF;
+    return A.X + ((int64_t)(A.t - 1) * A.N + j) * FF;
 }
 
 // Edge metadata and basis rows of one tile, by the 128 threads of a warpgroup: thread t
 // handles edge n = t % 64 and half of its K_P Gaussians.  u = r_i - r_j and d in double
 // (minimum image on periodic axes); bt_k = exp(-gamma (d - mu_k)^2) C(d) as fp16 (hi/lo);
-// zero for k >= K and for padding edges n >= ne.
-template <int KP, bool SPLIT>
+// zero for k >= K and for padding edges n >= ne.  Also the feature-row pointers of source
+// and destination used by the gathers (padding edges point at row 0, never used).
+template <int KP, bool SPLIT, int NW, bool BWD>
 __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char *R, int t, int i0, int i1, int ts,
                                               int ne)
 {
-    using S = TcSmem<KP, SPLIT>;
+    using S = TcSmem<KP, SPLIT, NW>;
     const int n = t & (TE - 1), half = t / TE;
-    int *sSrc = reinterpret_cast<int *>(R + S::SRC);
+    const float **sPx = reinterpret_cast<const float **>(R + S::PX);
+    const float **sPh = reinterpret_cast<const float **>(R + S::PH);
+    const float **sPxi = reinterpret_cast<const float **>(R + S::PXI);
+    const float **sPhi = reinterpret_cast<const float **>(R + S::PHI);
     int *sDst = reinterpret_cast<int *>(R + S::DST);
     double *sDist = reinterpret_cast<double *>(R + S::DIST);
     float *sU = reinterpret_cast<float *>(R + S::UVEC);
@@ -285,17 +314,26 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
         if (A.geo.periodic[2]) dz -= (double)A.geo.box[2] * rint(dz / (double)A.geo.box[2]);
         d = sqrt(dx * dx + dy * dy + dz * dz);
         if (half == 0) {
-            sSrc[n] = j;
             sDst[n] = i;
             sDist[n] = d;
-            sU[3 * n] = (float)(dx / d);
-            sU[3 * n + 1] = (float)(dy / d);
-            sU[3 * n + 2] = (float)(dz / d);
+            const double inv = 1.0 / d;
+            sU[3 * n] = (float)(dx * inv);
+            sU[3 * n + 1] = (float)(dy * inv);
+            sU[3 * n + 2] = (float)(dz * inv);
+        } else {
+            sPx[n] = feat_row(A, j);
+            if (BWD) {
+                sPh[n] = A.Hbar + (int64_t)j * FF;
+                sPxi[n] = feat_row(A, i);
+                sPhi[n] = A.Hbar + (int64_t)i * FF;
+            }
         }
     } else if (half == 0) {
-        sSrc[n] = -1;
         sDst[n] = -1;
         sDist[n] = 0.0;
+    } else {
+        sPx[n] = A.emb;
+        if (BWD) sPh[n] = sPxi[n] = sPhi[n] = A.emb;
     }
     const float C = 0.5f * (cospif((float)(d / A.basis.r_cut_d)) + 1.0f);
     unsigned char *Bh = R + S::B;
@@ -311,7 +349,7 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
             float b = 0.0f;
             if (n < ne && k < A.basis.K) {
                 const float x = (float)(d - A.basis.mu[k]);
-                b = expf(-A.basis.gamma * x * x) * C;
+                b = __expf(-A.basis.gamma * x * x) * C;
             }
             v[c] = b;
         }
@@ -320,10 +358,10 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
 }
 
 // D_A[f][n] = sum_k W1[f][k] bt[n][k]                          (M = 128, N = TE)
-template <int KP, bool SPLIT>
+template <int KP, bool SPLIT, int NW>
 __device__ __forceinline__ void issue_mma1(unsigned char *sm, unsigned char *R, uint32_t d)
 {
-    using S = TcSmem<KP, SPLIT>;
+    using S = TcSmem<KP, SPLIT, NW>;
     constexpr uint32_t ID = idesc_f16(128, TE, 0, 0);
     const uint32_t wh = smem_u32(sm + S::W1), wl = wh + S::W1B;
     const uint32_t bh = smem_u32(R + S::B), bl = bh + S::BB;
@@ -340,10 +378,10 @@ __device__ __forceinline__ void issue_mma1(unsigned char *sm, unsigned char *R, 
 
 // TRANS = false: D[o][n] = sum_i W2[o][i] T[n][i]   (forward filter layer 2)
 // TRANS = true : D[i][n] = sum_o W2[o][i] T[n][o]   (backward through layer 2)
-template <int KP, bool SPLIT, bool TRANS>
+template <int KP, bool SPLIT, int NW, bool TRANS>
 __device__ __forceinline__ void issue_mma_w2(unsigned char *sm, unsigned char *R, uint32_t d)
 {
-    using S = TcSmem<KP, SPLIT>;
+    using S = TcSmem<KP, SPLIT, NW>;
     constexpr uint32_t ID = idesc_f16(128, TE, TRANS ? 1 : 0, 1);
     const uint32_t wh = smem_u32(sm + S::W2), wl = wh + S::W2B;
     const uint32_t th = smem_u32(R + S::T), tl = th + S::TB;
@@ -361,10 +399,10 @@ __device__ __forceinline__ void issue_mma_w2(unsigned char *sm, unsigned char *R
 
 // D_G[n][k] = sum_f abar[n][f] W1[f][k]   (edges on M: M = TE = 64; row n of D sits in TMEM
 // lane (n % 16) + 32 (n / 16))
-template <int KP, bool SPLIT>
+template <int KP, bool SPLIT, int NW>
 __device__ __forceinline__ void issue_mma4(unsigned char *sm, unsigned char *R, uint32_t d)
 {
-    using S = TcSmem<KP, SPLIT>;
+    using S = TcSmem<KP, SPLIT, NW>;
     constexpr uint32_t ID = idesc_f16(TE, KP, 1, 1);
     const uint32_t wh = smem_u32(sm + S::W1), wl = wh + S::W1B;
     const uint32_t th = smem_u32(R + S::T), tl = th + S::TB;
@@ -380,23 +418,23 @@ __device__ __forceinline__ void issue_mma4(unsigned char *sm, unsigned char *R, 
 }
 
 // Kernel set-up: weights to shared memory, one mbarrier per warpgroup, TMEM for the CTA.
-template <int KP, bool SPLIT>
+template <int KP, bool SPLIT, int NW>
 __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm, int &skip)
 {
-    using S = TcSmem<KP, SPLIT>;
+    using S = TcSmem<KP, SPLIT, NW>;
     const int warp = threadIdx.x >> 5;
-    copy_to_smem(sm + S::W1, A.W1h, S::W1B);
-    copy_to_smem(sm + S::W2, A.W2h, S::W2B);
+    copy_to_smem<NW>(sm + S::W1, A.W1h, S::W1B);
+    copy_to_smem<NW>(sm + S::W2, A.W2h, S::W2B);
     if (SPLIT) {
-        copy_to_smem(sm + S::W1 + S::W1B, A.W1l, S::W1B);
-        copy_to_smem(sm + S::W2 + S::W2B, A.W2l, S::W2B);
+        copy_to_smem<NW>(sm + S::W1 + S::W1B, A.W1l, S::W1B);
+        copy_to_smem<NW>(sm + S::W2 + S::W2B, A.W2l, S::W2B);
     }
     if (threadIdx.x == 0) {
-        for (int g = 0; g < NWG; ++g) mbar_init(smem_u32(sm + S::GROUPS + g * S::REGION + S::MBAR), 1);
+        for (int g = 0; g < NW; ++g) mbar_init(smem_u32(sm + S::GROUPS + g * S::REGION + S::MBAR), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     }
-    if (warp == 0) tmem_alloc(smem_u32(sm + S::HOLD), TMEM_COLS);
+    if (warp == 0) tmem_alloc(smem_u32(sm + S::HOLD), 128 * NW);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -404,12 +442,13 @@ __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm
     return *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
 }
 
+template <int NW>
 __device__ __forceinline__ void teardown(uint32_t tmem)
 {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, TMEM_COLS);
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, 128 * NW);
 }
 
 // Per-warpgroup context: group g, thread t in group (= TMEM lane = feature), its shared region,
@@ -421,10 +460,10 @@ struct Group {
     int i0, i1;
 };
 
-template <int KP, bool SPLIT>
+template <int KP, bool SPLIT, int NW>
 __device__ __forceinline__ Group make_group(const EdgeTcArgs &A, unsigned char *sm, uint32_t tmem0)
 {
-    using S = TcSmem<KP, SPLIT>;
+    using S = TcSmem<KP, SPLIT, NW>;
     Group G;
     G.g = threadIdx.x / WGT;
     G.t = threadIdx.x % WGT;
@@ -432,7 +471,7 @@ __device__ __forceinline__ Group make_group(const EdgeTcArgs &A, unsigned char *
     G.mbar = smem_u32(G.R + S::MBAR);
     G.tm = tmem0 + (uint32_t)G.g * 128;
     G.lane = (uint32_t)((G.t >> 5) * 32) << 16;
-    const int p = blockIdx.x * NWG + G.g;
+    const int p = blockIdx.x * NW + G.g;
     G.i0 = A.part[p];
     G.i1 = A.part[p + 1];
     return G;
@@ -454,19 +493,33 @@ __device__ __forceinline__ bool mma_step(const Group &G, uint32_t &phase, int *d
     return wait_mma(G.g, G.mbar, phase, d_err);
 }
 
-template <int KP, bool SPLIT>
-__global__ void __launch_bounds__(NT, 1) k_edge_fwd_tc(EdgeTcArgs A)
+// s = ssp(a + b1) from TMEM columns [COL_A, COL_A + TE) into the activation tile
+template <bool SPLIT, int CH>
+__device__ __forceinline__ void ssp_to_tile(const Group &G, float b1f, unsigned char *Th, unsigned char *Tl)
 {
-    using S = TcSmem<KP, SPLIT>;
+#pragma unroll 1
+    for (int c = 0; c < TE / CH; ++c) {
+        float v[CH];
+        tmem_ld<CH>(G.tm + G.lane + COL_A + CH * c, v);
+#pragma unroll
+        for (int q = 0; q < CH; ++q) v[q] = ssp_fast(v[q] + b1f);
+        store_tile_col<SPLIT, CH>(Th, Tl, G.t, CH * c, v);
+    }
+}
+
+template <int KP, bool SPLIT, int NW, int CH>
+__global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
+{
+    using S = TcSmem<KP, SPLIT, NW>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
-    const uint32_t tmem0 = setup<KP, SPLIT>(A, sm, skip);
-    const Group G = make_group<KP, SPLIT>(A, sm, tmem0);
+    const uint32_t tmem0 = setup<KP, SPLIT, NW>(A, sm, skip);
+    const Group G = make_group<KP, SPLIT, NW>(A, sm, tmem0);
     const int f = G.t;
     if (!skip && G.i0 < G.i1) {
         const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
         const float b1f = A.b1[f], b2f = A.b2[f];
-        const int *sSrc = reinterpret_cast<const int *>(G.R + S::SRC);
+        const float *const *sPx = reinterpret_cast<const float *const *>(G.R + S::PX);
         const int *sDst = reinterpret_cast<const int *>(G.R + S::DST);
         unsigned char *Th = G.R + S::T, *Tl = Th + S::TB;
         uint32_t phase = 0;
@@ -475,38 +528,26 @@ __global__ void __launch_bounds__(NT, 1) k_edge_fwd_tc(EdgeTcArgs A)
         bool ok = true;
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT>(A, G.R, f, G.i0, G.i1, ts, ne);
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
-            // s = ssp(a + b1) into the activation tile
-#pragma unroll 1
-            for (int c = 0; c < TE / 32; ++c) {
-                float v[32];
-                tmem_ld32(G.tm + G.lane + COL_A + 32 * c, v);
-#pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] = ssp_fast(v[q] + b1f);
-                store_tile_col<SPLIT>(Th, Tl, f, 32 * c, v);
-            }
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
+            tile_prologue<KP, SPLIT, NW, false>(A, G.R, f, G.i0, G.i1, ts, ne);
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
+            ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, false>(sm, G.R, G.tm + COL_W); })))
                 break;
-            // h_i += x_src (.) (w + b2), segment sums per destination row
+            // h_i += x_src (.) (w + b2), running sums per destination row
 #pragma unroll 1
-            for (int c = 0; c < TE / 32; ++c) {
-                if (32 * c >= ne) break;
-                float v[32], xs[32];
-                tmem_ld32(G.tm + G.lane + COL_W + 32 * c, v);
+            for (int c = 0; c < TE / CH; ++c) {
+                if (CH * c >= ne) break;
+                float v[CH], xs[CH];
+                tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, v);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int n = 32 * c + q;
-                    xs[q] = n < ne ? featv(A.t, A.X, A.emb, A.types, A.N, sSrc[n], f) : 0.0f;
-                }
+                for (int q = 0; q < CH; ++q) xs[q] = __ldg(sPx[CH * c + q] + f);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int n = 32 * c + q;
+                for (int q = 0; q < CH; ++q) {
+                    const int n = CH * c + q;
                     if (n < ne) {
                         const int i = sDst[n];
                         if (i != cur) {
                             A.H[(int64_t)cur * FF + f] = hacc;
-                            for (int r = cur + 1; r < i; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
                             hacc = 0.0f;
                             cur = i;
                         }
@@ -519,10 +560,12 @@ __global__ void __launch_bounds__(NT, 1) k_edge_fwd_tc(EdgeTcArgs A)
         }
         if (ok) {
             A.H[(int64_t)cur * FF + f] = hacc;
-            for (int r = cur + 1; r < G.i1; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
+            // rows without edges receive no message
+            for (int r = G.i0; r < G.i1; ++r)
+                if (__ldg(A.row_ptr + r) == __ldg(A.row_ptr + r + 1)) A.H[(int64_t)r * FF + f] = 0.0f;
         }
     }
-    teardown(tmem0);
+    teardown<NW>(tmem0);
 }
 
 // Backward of one interaction block over the group's rows (see sn_ef_fp32.cu for the algebra):
@@ -530,19 +573,22 @@ __global__ void __launch_bounds__(NT, 1) k_edge_fwd_tc(EdgeTcArgs A)
 // wbar = x_j (.) hbar_i + x_i (.) hbar_j; sbar = W2^T wbar; abar = sbar (.) sigma(a);
 // btbar = W1^T abar (edges on M); dbar = btbar . d(bt)/dd; F_i -= dbar * u_ij / d_ij by the
 // row's owner only.  TMEM columns are reused: sbar overwrites w, btbar overwrites a.
-template <int KP, bool SPLIT>
-__global__ void __launch_bounds__(NT, 1) k_edge_bwd_tc(EdgeTcArgs A)
+template <int KP, bool SPLIT, int NW, int CH>
+__global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
 {
-    using S = TcSmem<KP, SPLIT>;
+    using S = TcSmem<KP, SPLIT, NW>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
-    const uint32_t tmem0 = setup<KP, SPLIT>(A, sm, skip);
-    const Group G = make_group<KP, SPLIT>(A, sm, tmem0);
+    const uint32_t tmem0 = setup<KP, SPLIT, NW>(A, sm, skip);
+    const Group G = make_group<KP, SPLIT, NW>(A, sm, tmem0);
     const int f = G.t;
     if (!skip && G.i0 < G.i1) {
         const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
         const float b1f = A.b1[f], b2f = A.b2[f];
-        const int *sSrc = reinterpret_cast<const int *>(G.R + S::SRC);
+        const float *const *sPx = reinterpret_cast<const float *const *>(G.R + S::PX);
+        const float *const *sPh = reinterpret_cast<const float *const *>(G.R + S::PH);
+        const float *const *sPxi = reinterpret_cast<const float *const *>(G.R + S::PXI);
+        const float *const *sPhi = reinterpret_cast<const float *const *>(G.R + S::PHI);
         const int *sDst = reinterpret_cast<const int *>(G.R + S::DST);
         const double *sDist = reinterpret_cast<const double *>(G.R + S::DIST);
         const float *sU = reinterpret_cast<const float *>(G.R + S::UVEC);
@@ -554,39 +600,27 @@ __global__ void __launch_bounds__(NT, 1) k_edge_bwd_tc(EdgeTcArgs A)
         bool ok = true;
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT>(A, G.R, f, G.i0, G.i1, ts, ne);
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
-#pragma unroll 1
-            for (int c = 0; c < TE / 32; ++c) {
-                float v[32];
-                tmem_ld32(G.tm + G.lane + COL_A + 32 * c, v);
-#pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] = ssp_fast(v[q] + b1f);
-                store_tile_col<SPLIT>(Th, Tl, f, 32 * c, v);
-            }
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
+            tile_prologue<KP, SPLIT, NW, true>(A, G.R, f, G.i0, G.i1, ts, ne);
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
+            ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, false>(sm, G.R, G.tm + COL_W); })))
                 break;
-            // xbar and wbar; source and destination features of a chunk are loaded up front
+            // xbar and wbar; source and destination features of a chunk loaded up front
 #pragma unroll 1
-            for (int c = 0; c < TE / 32; ++c) {
-                float w[32], hb[32], xj[32], hi_[32], xi_[32];
-                tmem_ld32(G.tm + G.lane + COL_W + 32 * c, w);
+            for (int c = 0; c < TE / CH; ++c) {
+                float w[CH], hb[CH], xj[CH], hi_[CH], xi_[CH];
+                tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, w);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int n = 32 * c + q;
-                    if (n < ne) {
-                        const int j = sSrc[n], i = sDst[n];
-                        hb[q] = __ldg(A.Hbar + (int64_t)j * FF + f);
-                        xj[q] = featv(A.t, A.X, A.emb, A.types, A.N, j, f);
-                        hi_[q] = __ldg(A.Hbar + (int64_t)i * FF + f);
-                        xi_[q] = featv(A.t, A.X, A.emb, A.types, A.N, i, f);
-                    } else {
-                        hb[q] = xj[q] = hi_[q] = xi_[q] = 0.0f;
-                    }
+                for (int q = 0; q < CH; ++q) {
+                    const int n = CH * c + q;
+                    hb[q] = __ldg(sPh[n] + f);
+                    xj[q] = __ldg(sPx[n] + f);
+                    hi_[q] = __ldg(sPhi[n] + f);
+                    xi_[q] = __ldg(sPxi[n] + f);
                 }
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int n = 32 * c + q;
+                for (int q = 0; q < CH; ++q) {
+                    const int n = CH * c + q;
                     if (n < ne) {
                         const int i = sDst[n];
                         if (i != cur) {
@@ -599,21 +633,21 @@ __global__ void __launch_bounds__(NT, 1) k_edge_bwd_tc(EdgeTcArgs A)
                     }
                     xj[q] = n < ne ? xj[q] * hi_[q] + xi_[q] * hb[q] : 0.0f;
                 }
-                store_tile_col<SPLIT>(Th, Tl, f, 32 * c, xj);
+                store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, xj);
             }
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, true>(sm, G.R, G.tm + COL_W); })))
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, true>(sm, G.R, G.tm + COL_W); })))
                 break;
             // abar = sbar (.) sigma(a + b1)
 #pragma unroll 1
-            for (int c = 0; c < TE / 32; ++c) {
-                float sb[32], a[32];
-                tmem_ld32(G.tm + G.lane + COL_W + 32 * c, sb);
-                tmem_ld32(G.tm + G.lane + COL_A + 32 * c, a);
+            for (int c = 0; c < TE / CH; ++c) {
+                float sb[CH], a[CH];
+                tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, sb);
+                tmem_ld<CH>(G.tm + G.lane + COL_A + CH * c, a);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) sb[q] *= sigmoid_fast(a[q] + b1f);
-                store_tile_col<SPLIT>(Th, Tl, f, 32 * c, sb);
+                for (int q = 0; q < CH; ++q) sb[q] *= sigmoid_fast(a[q] + b1f);
+                store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, sb);
             }
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma4<KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma4<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
             // lanes 0-15 of each warp quadrant: edge n = 16 * quadrant + lane, dbar and force
             {
                 const int l = f & 31, n = (f >> 5) * 16 + l;
@@ -624,15 +658,15 @@ __global__ void __launch_bounds__(NT, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 const float C = 0.5f * (cospif(ratio) + 1.0f);
                 const float dC = -0.5f * (float)M_PI / A.basis.r_cut * sinpif(ratio);
 #pragma unroll 1
-                for (int c = 0; c < KP / 32; ++c) {
-                    float gg[32];
-                    tmem_ld32(G.tm + G.lane + COL_A + 32 * c, gg);
+                for (int c = 0; c < KP / CH; ++c) {
+                    float gg[CH];
+                    tmem_ld<CH>(G.tm + G.lane + COL_A + CH * c, gg);
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        const int k = 32 * c + q;
+                    for (int q = 0; q < CH; ++q) {
+                        const int k = CH * c + q;
                         if (mine && k < A.basis.K) {
                             const float x = (float)(d - A.basis.mu[k]);
-                            const float phi = expf(-A.basis.gamma * x * x);
+                            const float phi = __expf(-A.basis.gamma * x * x);
                             gsum = fmaf(gg[q], -2.0f * A.basis.gamma * x * phi * C + phi * dC, gsum);
                         }
                     }
@@ -662,7 +696,7 @@ __global__ void __launch_bounds__(NT, 1) k_edge_bwd_tc(EdgeTcArgs A)
         }
         if (ok && cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
     }
-    teardown(tmem0);
+    teardown<NW>(tmem0);
 }
 
 template <typename Kern>
@@ -671,31 +705,38 @@ cudaError_t prepare(Kern k, uint32_t bytes)
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <int KP, bool SPLIT>
+template <int KP, bool SPLIT, int NW, int CH>
 cudaError_t launch_t(const EdgeTcArgs &a, bool backward, int G, cudaStream_t s)
 {
-    using S = TcSmem<KP, SPLIT>;
+    using S = TcSmem<KP, SPLIT, NW>;
     static_assert(S::BYTES <= 227 * 1024, "shared memory plan exceeds 227 KB");
+    static_assert(NW == 2 || NW == 4, "TMEM allocations are powers of two: 2 or 4 groups");
     cudaError_t e;
     if (backward) {
-        if ((e = prepare(k_edge_bwd_tc<KP, SPLIT>, S::BYTES))) return e;
-        k_edge_bwd_tc<KP, SPLIT><<<G, NT, S::BYTES, s>>>(a);
+        if ((e = prepare(k_edge_bwd_tc<KP, SPLIT, NW, CH>, S::BYTES))) return e;
+        k_edge_bwd_tc<KP, SPLIT, NW, CH><<<G, WGT * NW, S::BYTES, s>>>(a);
     } else {
-        if ((e = prepare(k_edge_fwd_tc<KP, SPLIT>, S::BYTES))) return e;
-        k_edge_fwd_tc<KP, SPLIT><<<G, NT, S::BYTES, s>>>(a);
+        if ((e = prepare(k_edge_fwd_tc<KP, SPLIT, NW, CH>, S::BYTES))) return e;
+        k_edge_fwd_tc<KP, SPLIT, NW, CH><<<G, WGT * NW, S::BYTES, s>>>(a);
     }
     return cudaGetLastError();
 }
 
+// The split (fp32-accurate) mode holds two fp16 copies of every operand: two warpgroups fit in
+// shared memory.  The fp16 mode runs four (16 warps per SM), with 16-column chunks to stay
+// within 128 registers per thread.
+constexpr int groups_for(bool split) { return split ? 2 : 4; }
+
 }  // namespace
 
-int tc_groups_per_cta() { return NWG; }
+int tc_groups_per_cta(bool split) { return groups_for(split); }
 
-// G CTAs, each running NWG independent row ranges: a.part must hold G * NWG + 1 entries.
+// G CTAs, each running tc_groups_per_cta(split) independent row ranges: a.part must hold
+// G * tc_groups_per_cta(split) + 1 entries.
 cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s)
 {
-    if (KP == 64) return split ? launch_t<64, true>(a, backward, G, s) : launch_t<64, false>(a, backward, G, s);
-    if (KP == 32) return split ? launch_t<32, true>(a, backward, G, s) : launch_t<32, false>(a, backward, G, s);
+    if (KP == 64) return split ? launch_t<64, true, 2, 32>(a, backward, G, s) : launch_t<64, false, 4, 16>(a, backward, G, s);
+    if (KP == 32) return split ? launch_t<32, true, 2, 32>(a, backward, G, s) : launch_t<32, false, 4, 16>(a, backward, G, s);
     return cudaErrorInvalidValue;
 }
 

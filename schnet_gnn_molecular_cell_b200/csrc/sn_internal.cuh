@@ -158,7 +158,7 @@ struct EdgeTcArgs {
 };
 
 cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s);
-int tc_groups_per_cta();   // independent row ranges per CTA of the tensor-core edge kernels
+int tc_groups_per_cta(bool split);   // independent row ranges per CTA of the tensor-core edge kernels
 void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, uint16_t *hi, uint16_t *lo);
 
 // ---------------------------------------------------------------- integrator
