@@ -54,9 +54,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--precision", default="tc32", choices=list(PRECISIONS),
-                    help="filter-network arithmetic: tc32 = fp32-accurate fp16-split on tensor cores "
-                         "(default), fp16 = single fp16 operands (W16A16), fp32 = CUDA cores")
+    ap.add_argument("--precision", default="fp16", choices=list(PRECISIONS),
+                    help="network arithmetic: fp16 = fp16 operands on tensor cores, fp32 accumulate "
+                         "(W16A16, default), tc32 = fp32-accurate fp16 split on tensor cores, fp32 = CUDA cores")
     ap.add_argument("--no-variants", action="store_true", help="skip the short runs of the other precisions")
     return ap.parse_args()
 

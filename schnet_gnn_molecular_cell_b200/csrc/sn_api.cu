@@ -340,15 +340,22 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
 
     // fp16 hi/lo copies of W1 and W2 in the tensor-core operand layout (per block: W1h W1l W2h W2l)
     std::vector<uint16_t> tcw;
-    const size_t n_w1 = (size_t)F * KP, n_w2 = (size_t)F * F, per_tc = 2 * n_w1 + 2 * n_w2;
+    // per block: W1 hi, lo, W2 hi, lo, U1 hi, lo, U2 hi, lo; then R1 (padded to F rows) hi, lo
+    const size_t n_w1 = (size_t)F * KP, n_w2 = (size_t)F * F, per_tc = 2 * n_w1 + 6 * n_w2;
     if (cfg->precision != SN_PREC_FP32) {
-        tcw.assign(per_tc * T, 0);
+        tcw.assign(per_tc * T + 2 * n_w2, 0);
         for (int t = 0; t < T; ++t) {
             const float *blk = weights_host + (int64_t)NT * F + t * per_block;
             uint16_t *o = tcw.data() + per_tc * t;
+            const float *W2 = blk + (int64_t)F * K + F, *U1 = W2 + (int64_t)F * F + F, *U2 = U1 + (int64_t)F * F + F;
             sn::tc_pack_matrix(blk, F, K, KP, o, o + n_w1);
-            sn::tc_pack_matrix(blk + (int64_t)F * K + F, F, F, F, o + 2 * n_w1, o + 2 * n_w1 + n_w2);
+            sn::tc_pack_matrix(W2, F, F, F, o + 2 * n_w1, o + 2 * n_w1 + n_w2);
+            sn::tc_pack_matrix(U1, F, F, F, o + 2 * n_w1 + 2 * n_w2, o + 2 * n_w1 + 3 * n_w2);
+            sn::tc_pack_matrix(U2, F, F, F, o + 2 * n_w1 + 4 * n_w2, o + 2 * n_w1 + 5 * n_w2);
         }
+        const float *R1 = weights_host + (int64_t)NT * F + T * per_block;
+        uint16_t *o = tcw.data() + per_tc * T;
+        sn::tc_pack_matrix(R1, H, F, F, o, o + n_w2);   // rows H..F-1 stay zero
     }
 
     cudaError_t e = cudaMalloc(&ctx->d_weights, sizeof(float) * pk.buf.size());
@@ -395,12 +402,20 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
             m.blk[t].W1l = o + n_w1;
             m.blk[t].W2h = o + 2 * n_w1;
             m.blk[t].W2l = o + 2 * n_w1 + n_w2;
+            m.blk[t].U1h = o + 2 * n_w1 + 2 * n_w2;
+            m.blk[t].U1l = o + 2 * n_w1 + 3 * n_w2;
+            m.blk[t].U2h = o + 2 * n_w1 + 4 * n_w2;
+            m.blk[t].U2l = o + 2 * n_w1 + 5 * n_w2;
         }
     }
     m.ro.R1 = W + o_R1;
     m.ro.e1 = W + o_e1;
     m.ro.R2 = W + o_R2;
     m.ro.e2 = W + o_e2;
+    if (ctx->d_tcw) {
+        m.ro.R1h = ctx->d_tcw + per_tc * T;
+        m.ro.R1l = ctx->d_tcw + per_tc * T + n_w2;
+    }
     *out = ctx;
     return SN_OK;
 }

@@ -655,12 +655,67 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
     const int64_t n_tiles = (N + NA - 1) / NA;
     const unsigned node_grid = (unsigned)(n_tiles < n_sm ? (n_tiles < 1 ? 1 : n_tiles) : n_sm);
 
+    if (m.precision != SN_PREC_FP32) {
+        // tensor-core precisions: edge and node networks on tcgen05
+        const bool split = m.precision == SN_PREC_TC32;
+        NodeTcArgs nt{};
+        nt.types = types;
+        nt.emb = m.emb;
+        nt.X = w.x;
+        nt.P = w.p;
+        nt.H = w.h;
+        nt.Hbar = w.hbar;
+        nt.Xbar = w.xbar;
+        nt.eps = w.eps;
+        nt.forces = forces;
+        nt.N = N;
+        nt.R1h = m.ro.R1h;
+        nt.R1l = m.ro.R1l;
+        nt.e1 = m.ro.e1;
+        nt.R2 = m.ro.R2;
+        nt.e2 = m.ro.e2;
+        nt.d_err = d_err;
+        auto node_args = [&](int t) {
+            NodeTcArgs a = nt;
+            a.t = t;
+            a.U1h = m.blk[t].U1h;
+            a.U1l = m.blk[t].U1l;
+            a.U2h = m.blk[t].U2h;
+            a.U2l = m.blk[t].U2l;
+            a.c1 = m.blk[t].c1;
+            a.c2 = m.blk[t].c2;
+            return a;
+        };
+        for (int t = 0; t < m.T; ++t) {
+            ea.w = m.blk[t];
+            ea.t = t;
+            trace_begin(tr, KK_EDGE_FWD, s);
+            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err), KP, split, false, w.G, s))) return e;
+            trace_end(tr, s);
+            trace_begin(tr, KK_NODE_FWD, s);
+            if ((e = launch_node_tc(node_args(t), split, 0, n_sm, s))) return e;
+            trace_end(tr, s);
+        }
+        trace_begin(tr, KK_NODE_FWD, s);
+        if ((e = launch_node_tc(node_args(m.T - 1), split, 1, n_sm, s))) return e;   // readout of x^T
+        trace_end(tr, s);
+        for (int t = m.T - 1; t >= 0; --t) {
+            trace_begin(tr, KK_NODE_BWD, s);
+            if ((e = launch_node_tc(node_args(t), split, 2, n_sm, s))) return e;     // hbar^t
+            trace_end(tr, s);
+            ea.w = m.blk[t];
+            ea.t = t;
+            trace_begin(tr, KK_EDGE_BWD, s);
+            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err), KP, split, true, w.G, s))) return e;
+            trace_end(tr, s);
+        }
+        return cudaGetLastError();
+    }
     for (int t = 0; t < m.T; ++t) {
         ea.w = m.blk[t];
         ea.t = t;
         trace_begin(tr, KK_EDGE_FWD, s);
-        if (m.precision == SN_PREC_FP32) k_edge_fwd<F, KP><<<w.G, F, fwd_bytes, s>>>(ea);
-        else if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err), KP, m.precision == SN_PREC_TC32, false, w.G, s))) return e;
+        k_edge_fwd<F, KP><<<w.G, F, fwd_bytes, s>>>(ea);
         trace_end(tr, s);
         na.w = m.blk[t];
         na.t = t;
@@ -673,8 +728,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
         ea.w = m.blk[t];
         ea.t = t;
         trace_begin(tr, KK_EDGE_BWD, s);
-        if (m.precision == SN_PREC_FP32) k_edge_bwd<F, KP><<<w.G, F, bwd_bytes, s>>>(ea);
-        else if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err), KP, m.precision == SN_PREC_TC32, true, w.G, s))) return e;
+        k_edge_bwd<F, KP><<<w.G, F, bwd_bytes, s>>>(ea);
         trace_end(tr, s);
         if (t > 0) {
             na.w = m.blk[t - 1];

@@ -26,207 +26,18 @@
 #include <math.h>
 
 #include "sn_internal.cuh"
+#include "sn_tc_common.cuh"
 
 namespace sn {
 
 namespace {
 
+using namespace tc;
+
 constexpr int TE = 64;           // edges per tile
-constexpr int WGT = 128;         // threads per warpgroup (thread t of a group <-> TMEM lane t)
-constexpr int FF = 128;          // feature width supported by these kernels
 // TMEM: 128 columns per warpgroup (128 * NW per CTA)
 // per-warpgroup TMEM columns: a (and later btbar) in [0, 64), w (and later sbar) in [64, 128)
 constexpr uint32_t COL_A = 0, COL_W = 64;
-constexpr float LN2F = 0.693147180559945309f;
-
-// ------------------------------------------------------------------ PTX wrappers (sm_100a)
-__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void tmem_alloc(uint32_t holder, uint32_t ncols)
-{
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(holder), "r"(ncols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
-{
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
-        : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint32_t mbar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mbar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(mbar), "r"(parity)
-        : "memory");
-    return ok;
-}
-
-// This lane's 32 consecutive 32-bit TMEM columns starting at taddr (warp w reads lanes 32w..).
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
-{
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// This lane's 16 consecutive 32-bit TMEM columns starting at taddr.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
-{
-    uint32_t r[16];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-template <int CH>
-__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[CH])
-{
-    if constexpr (CH == 32) tmem_ld32(taddr, v);
-    else tmem_ld16(taddr, v);
-}
-
-// Shared-memory matrix descriptor, no swizzle (layout type 0), version 1.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
-{
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
-}
-
-// Instruction descriptor for kind::f16: fp16 A and B, fp32 D, dense.
-constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major)
-{
-    return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
-           ((uint32_t)(M >> 4) << 24);
-}
-
-// ------------------------------------------------------------------ helpers
-
-__device__ __forceinline__ int row_of_edge(const int32_t *__restrict__ row_ptr, int i0, int i1, int e)
-{
-    int lo = i0, hi = i1 - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (__ldg(row_ptr + mid) <= e) lo = mid;
-        else hi = mid - 1;
-    }
-    return lo;
-}
-
-
-// 8 values -> one 16-byte fp16 run (hi) and, for SPLIT, the run of residuals (lo)
-template <bool SPLIT>
-__device__ __forceinline__ void store8(unsigned char *hi, unsigned char *lo, uint32_t off, const float *v)
-{
-    __half2 h[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) h[q] = __floats2half2_rn(v[2 * q], v[2 * q + 1]);
-    *reinterpret_cast<uint4 *>(hi + off) = make_uint4(*reinterpret_cast<uint32_t *>(&h[0]), *reinterpret_cast<uint32_t *>(&h[1]),
-                                                      *reinterpret_cast<uint32_t *>(&h[2]), *reinterpret_cast<uint32_t *>(&h[3]));
-    if (SPLIT) {
-        __half2 l[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const float2 b = __half22float2(h[q]);
-            l[q] = __floats2half2_rn(v[2 * q] - b.x, v[2 * q + 1] - b.y);
-        }
-        *reinterpret_cast<uint4 *>(lo + off) = make_uint4(*reinterpret_cast<uint32_t *>(&l[0]), *reinterpret_cast<uint32_t *>(&l[1]),
-                                                          *reinterpret_cast<uint32_t *>(&l[2]), *reinterpret_cast<uint32_t *>(&l[3]));
-    }
-}
-
-// Activation tile T[n][f] (edges n contiguous in 16-byte runs): element (n, f) at
-// (n % 8) * 2 + (n / 8) * 2048 + (f % 8) * 16 + (f / 8) * 128.  Thread f stores edges
-// n0 .. n0+31 of its feature.  TE = 64 edges: 16 KB per fp16 copy.
-template <bool SPLIT, int CH>
-__device__ __forceinline__ void store_tile_col(unsigned char *Th, unsigned char *Tl, int f, int n0, const float (&v)[CH])
-{
-    const uint32_t base = (uint32_t)((f & 7) * 16 + (f >> 3) * 128);
-#pragma unroll
-    for (int g = 0; g < CH / 8; ++g) store8<SPLIT>(Th, Tl, base + (uint32_t)(((n0 >> 3) + g) * 2048), v + 8 * g);
-}
-
-// Named barrier of one warpgroup (ids 1..4; id 0 is __syncthreads).
-__device__ __forceinline__ void wg_sync(int g)
-{
-    asm volatile("bar.sync %0, %1;" ::"r"(g + 1), "r"(WGT) : "memory");
-}
-
-// Warpgroup barrier that also returns whether every thread passed a true predicate.
-__device__ __forceinline__ int wg_sync_and(int g, int pred)
-{
-    int out;
-    asm volatile(
-        "{\n\t.reg .pred q, p;\n\tsetp.ne.s32 q, %1, 0;\n\t"
-        "bar.red.and.pred p, %2, %3, q;\n\tselp.s32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(out)
-        : "r"(pred), "r"(g + 1), "r"(WGT)
-        : "memory");
-    return out;
-}
-
-// Bounded wait for the MMAs committed to a warpgroup's mbarrier; every thread of the group
-// calls it at the same point.  On a time-out (never expected: nothing here waits on another
-// agent) the error bit is set and the whole group returns false.
-__device__ __forceinline__ bool wait_mma(int g, uint32_t mbar, uint32_t &phase, int *d_err)
-{
-    const long long t0 = clock64();
-    int ok = 0;
-    for (;;) {
-        if (mbar_try_wait(mbar, phase)) {
-            ok = 1;
-            break;
-        }
-        if (clock64() - t0 > (1ll << 33)) break;
-    }
-    phase ^= 1u;
-    ok = wg_sync_and(g, ok);
-    if (!ok && (threadIdx.x % WGT) == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
-    tc_fence_after();
-    return ok != 0;
-}
 
 // Shared-memory plan (bytes): weights shared by the CTA, then one region per warpgroup.
 template <int KP, bool SPLIT, int NW>
@@ -263,11 +74,16 @@ struct TcSmem {
 
 namespace {
 
-// Activations with the hardware exp2/log2 units (__expf, __logf): ssp(x) = max(x, 0) +
-// ln(1 + e^-|x|) - ln 2 and sigma(x) = 1 / (1 + e^-x).  Absolute error ~3e-7, below the
-// 2^-22 resolution of the split fp16 operands they feed.
-__device__ __forceinline__ float ssp_fast(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))) - LN2F; }
-__device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
+__device__ __forceinline__ int row_of_edge(const int32_t *__restrict__ row_ptr, int i0, int i1, int e)
+{
+    int lo = i0, hi = i1 - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (__ldg(row_ptr + mid) <= e) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
 
 template <int NW>
 __device__ __forceinline__ void copy_to_smem(unsigned char *dst, const void *src, uint32_t bytes)

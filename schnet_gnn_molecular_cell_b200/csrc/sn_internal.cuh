@@ -61,9 +61,9 @@ struct BlockW {
     const float *c1;   // [F]
     const float *U2;   // [F][F+1]
     const float *c2;   // [F]
-    // tensor-core precisions: W1 and W2 as fp16 hi / lo in the core-matrix layout of
+    // tensor-core precisions: W1, W2, U1, U2 as fp16 hi / lo in the core-matrix layout of
     // sn_ef_tc.cu (lo = fp16(w - hi), used by the split mode)
-    const void *W1h, *W1l, *W2h, *W2l;
+    const void *W1h, *W1l, *W2h, *W2l, *U1h, *U1l, *U2h, *U2l;
 };
 
 struct ReadoutW {
@@ -71,6 +71,7 @@ struct ReadoutW {
     const float *e1;   // [H]
     const float *R2;   // [H]
     const float *e2;   // [1]
+    const void *R1h, *R1l;   // tensor-core precisions: R1 padded to 128 rows, fp16 hi / lo
 };
 
 struct Geometry {
@@ -160,6 +161,27 @@ struct EdgeTcArgs {
 cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s);
 int tc_groups_per_cta(bool split);   // independent row ranges per CTA of the tensor-core edge kernels
 void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, uint16_t *hi, uint16_t *lo);
+
+// Arguments of the tensor-core node kernels (F = 128).
+struct NodeTcArgs {
+    const int32_t *types;
+    const float *emb;
+    float *X;          // [T][N][F]
+    float *P;          // [T][N][F]
+    const float *H;    // [N][F]
+    float *Hbar;       // [N][F]
+    float *Xbar;       // [N][F]
+    float *eps;        // [N]
+    float *forces;     // [N][3]
+    int64_t N;
+    int t;
+    const void *U1h, *U1l, *U2h, *U2l, *R1h, *R1l;
+    const float *c1, *c2, *e1, *R2, *e2;
+    int *d_err;
+};
+
+// which: 0 update of block a.t, 1 readout of x^T = X[a.t], 2 backward of block a.t's update
+cudaError_t launch_node_tc(const NodeTcArgs &a, bool split, int which, int n_sm, cudaStream_t s);
 
 // ---------------------------------------------------------------- integrator
 cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t n3, float c,

@@ -1,0 +1,332 @@
+// Node (per-atom) networks on the tensor cores: the update network with its residual, the
+// readout, and the backward of the update network (FlashSchNet §3.2 "update network with
+// residual connection", "Energy readout"; §4.4 applies W16A16 to the update and readout
+// networks as well as the filter network).  Per tile of TA = 128 atoms, with feature f =
+// TMEM lane f and atoms on the MMA N dimension:
+//   update   D_P = U1 h^T, p = D_P + c1;  D_Y = U2 ssp(p)^T, x^{t+1} = x^t + D_Y + c2
+//   readout  D_O = R1 x^T (R1 padded to 128 rows), o = D_O + e1; eps = R2 . ssp(o) + e2;
+//            obar = R2 (.) sigma(o); D_X = R1^T obar, xbar^T = D_X
+//   backward D_Q = U2^T xbar, pbar = D_Q (.) sigma(p);  D_H = U1^T pbar, hbar = D_H
+// Operands and precision modes as in sn_ef_tc.cu (fp16, or fp16 hi/lo split).
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "sn_internal.cuh"
+#include "sn_tc_common.cuh"
+
+namespace sn {
+
+namespace {
+
+using namespace tc;
+
+constexpr int TA = 128;          // atoms per tile (MMA N)
+
+template <bool SPLIT>
+struct NodeSmem {
+    static constexpr int NS = SPLIT ? 2 : 1;
+    static constexpr uint32_t WB = FF * FF * 2;     // one fp16 copy of a 128 x 128 weight
+    static constexpr uint32_t TB = TA * FF * 2;     // activation tile
+    static constexpr uint32_t W0 = 0;               // first weight (hi, lo)
+    static constexpr uint32_t W1 = W0 + NS * WB;    // second weight (hi, lo)
+    static constexpr uint32_t T = W1 + NS * WB;
+    static constexpr uint32_t MBAR = T + NS * TB;   // uint64
+    static constexpr uint32_t HOLD = MBAR + 8;      // TMEM address
+    static constexpr uint32_t PR = HOLD + 8;        // float[64][TA] readout products (readout only)
+    static constexpr uint32_t BYTES_UPDATE = PR;
+    static constexpr uint32_t BYTES_READOUT = PR + 64 * TA * 4;
+};
+
+__device__ __forceinline__ void copy_block(unsigned char *dst, const void *src, uint32_t bytes)
+{
+    const uint4 *s = reinterpret_cast<const uint4 *>(src);
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+    for (uint32_t q = threadIdx.x; q < bytes / 16; q += WGT) d[q] = __ldg(s + q);
+}
+
+// D[o][a] = sum_i W[o][i] T[a][i]  (TRANS = false)  or  D[i][a] = sum_o W[o][i] T[a][o]  (TRANS)
+template <bool SPLIT, bool TRANS>
+__device__ __forceinline__ void issue_gemm(unsigned char *W, unsigned char *T, uint32_t d)
+{
+    using S = NodeSmem<SPLIT>;
+    constexpr uint32_t ID = idesc_f16(128, TA, TRANS ? 1 : 0, 1);
+    const uint32_t wh = smem_u32(W), wl = wh + S::WB;
+    const uint32_t th = smem_u32(T), tl = th + S::TB;
+    const uint32_t a_lbo = TRANS ? 2048 : 128, a_sbo = TRANS ? 128 : 2048, a_step = TRANS ? 4096 : 256;
+#pragma unroll
+    for (int j = 0; j < FF / 16; ++j) {
+        const uint32_t oa = (uint32_t)j * a_step, ob = (uint32_t)j * 256;
+        mma_f16(d, sdesc(wh + oa, a_lbo, a_sbo), sdesc(th + ob, 128, 2048), ID, j > 0);
+        if (SPLIT) {
+            mma_f16(d, sdesc(wh + oa, a_lbo, a_sbo), sdesc(tl + ob, 128, 2048), ID, 1);
+            mma_f16(d, sdesc(wl + oa, a_lbo, a_sbo), sdesc(th + ob, 128, 2048), ID, 1);
+        }
+    }
+}
+
+template <bool SPLIT, bool TRANS>
+__device__ __forceinline__ bool gemm_step(unsigned char *W, unsigned char *T, uint32_t d, uint32_t mbar,
+                                          uint32_t &phase, int *d_err)
+{
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        tc_fence_after();
+        issue_gemm<SPLIT, TRANS>(W, T, d);
+        mma_commit(mbar);
+    }
+    return wait_mma(0, mbar, phase, d_err);
+}
+
+// value(a) for the 128 atoms of the tile at column f, into the activation tile (zero past N)
+template <bool SPLIT, typename Get>
+__device__ __forceinline__ void tile_from(unsigned char *T, int f, int64_t a0, int64_t N, Get get)
+{
+    using S = NodeSmem<SPLIT>;
+#pragma unroll 1
+    for (int c = 0; c < TA / 32; ++c) {
+        float v[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const int64_t a = a0 + 32 * c + q;
+            v[q] = a < N ? get(a) : 0.0f;
+        }
+        store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
+    }
+}
+
+__device__ __forceinline__ const float *x_row(const NodeTcArgs &A, int t, int64_t a)
+{
+    if (t == 0) return A.emb + (int64_t)__ldg(A.types + a) * FF;
+    return A.X + ((int64_t)(t - 1) * A.N + a) * FF;
+}
+
+template <bool SPLIT>
+__device__ __forceinline__ uint32_t node_setup(const NodeTcArgs &A, unsigned char *sm, const void *w0h,
+                                               const void *w0l, const void *w1h, const void *w1l, int &skip)
+{
+    using S = NodeSmem<SPLIT>;
+    copy_block(sm + S::W0, w0h, S::WB);
+    if (SPLIT) copy_block(sm + S::W0 + S::WB, w0l, S::WB);
+    if (w1h) {
+        copy_block(sm + S::W1, w1h, S::WB);
+        if (SPLIT) copy_block(sm + S::W1 + S::WB, w1l, S::WB);
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(sm + S::MBAR), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
+    }
+    if ((threadIdx.x >> 5) == 0) tmem_alloc(smem_u32(sm + S::HOLD), 256);
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    return *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
+}
+
+__device__ __forceinline__ void node_teardown(uint32_t tmem)
+{
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if ((threadIdx.x >> 5) == 0) tmem_dealloc(tmem, 256);
+}
+
+// p = U1 h + c1 (saved); x^{t+1} = x^t + U2 ssp(p) + c2
+template <bool SPLIT>
+__global__ void __launch_bounds__(WGT, 1) k_node_update_tc(NodeTcArgs A)
+{
+    using S = NodeSmem<SPLIT>;
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ int skip;
+    const uint32_t tmem = node_setup<SPLIT>(A, sm, A.U1h, A.U1l, A.U2h, A.U2l, skip);
+    const int f = threadIdx.x;
+    const uint32_t lane = (uint32_t)((f >> 5) * 32) << 16;
+    const uint32_t mbar = smem_u32(sm + S::MBAR);
+    uint32_t phase = 0;
+    const int64_t n_tiles = (A.N + TA - 1) / TA;
+    if (!skip) {
+        const float c1f = A.c1[f], c2f = A.c2[f];
+        unsigned char *T = sm + S::T;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const int64_t a0 = tile * TA;
+            tile_from<SPLIT>(T, f, a0, A.N, [&](int64_t a) { return A.H[a * FF + f]; });
+            if (!gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err)) break;
+#pragma unroll 1
+            for (int c = 0; c < TA / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int64_t a = a0 + 32 * c + q;
+                    v[q] += c1f;
+                    if (a < A.N) A.P[((int64_t)A.t * A.N + a) * FF + f] = v[q];
+                    v[q] = ssp_fast(v[q]);
+                }
+                store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
+            }
+            if (!gemm_step<SPLIT, false>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err)) break;
+#pragma unroll 1
+            for (int c = 0; c < TA / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane + 128 + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int64_t a = a0 + 32 * c + q;
+                    if (a < A.N) A.X[((int64_t)A.t * A.N + a) * FF + f] = __ldg(x_row(A, A.t, a) + f) + v[q] + c2f;
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+        }
+    }
+    node_teardown(tmem);
+}
+
+// o = R1 x^T + e1; eps = R2 . ssp(o) + e2; xbar^T = R1^T (R2 (.) sigma(o)); forces = 0
+template <bool SPLIT>
+__global__ void __launch_bounds__(WGT, 1) k_node_readout_tc(NodeTcArgs A)
+{
+    using S = NodeSmem<SPLIT>;
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ int skip;
+    const uint32_t tmem = node_setup<SPLIT>(A, sm, A.R1h, A.R1l, nullptr, nullptr, skip);
+    const int f = threadIdx.x;
+    const uint32_t lane = (uint32_t)((f >> 5) * 32) << 16;
+    const uint32_t mbar = smem_u32(sm + S::MBAR);
+    float *sPr = reinterpret_cast<float *>(sm + S::PR);
+    uint32_t phase = 0;
+    const int64_t n_tiles = (A.N + TA - 1) / TA;
+    const int H = FF / 2;
+    if (!skip) {
+        const float e1k = f < H ? A.e1[f] : 0.0f, r2k = f < H ? A.R2[f] : 0.0f, e2 = A.e2[0];
+        unsigned char *T = sm + S::T;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const int64_t a0 = tile * TA;
+            tile_from<SPLIT>(T, f, a0, A.N, [&](int64_t a) { return A.X[((int64_t)(A.t) * A.N + a) * FF + f]; });
+            if (!gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err)) break;
+#pragma unroll 1
+            for (int c = 0; c < TA / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const float o = v[q] + e1k;
+                    if (f < H) sPr[f * TA + 32 * c + q] = r2k * ssp_fast(o);
+                    v[q] = f < H ? r2k * sigmoid_fast(o) : 0.0f;
+                }
+                store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
+            }
+            if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem + 128, mbar, phase, A.d_err)) break;
+            {   // per-atom energy (fixed summation order) and zero forces
+                const int64_t a = a0 + f;
+                if (a < A.N) {
+                    float e = e2;
+                    for (int k = 0; k < H; ++k) e += sPr[k * TA + f];
+                    A.eps[a] = e;
+                    A.forces[a * 3] = 0.0f;
+                    A.forces[a * 3 + 1] = 0.0f;
+                    A.forces[a * 3 + 2] = 0.0f;
+                }
+            }
+#pragma unroll 1
+            for (int c = 0; c < TA / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane + 128 + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int64_t a = a0 + 32 * c + q;
+                    if (a < A.N) A.Xbar[a * FF + f] = v[q];
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+        }
+    }
+    node_teardown(tmem);
+}
+
+// hbar = U1^T (sigma(p) (.) U2^T xbar)   (block t's update network, p = P[t])
+template <bool SPLIT>
+__global__ void __launch_bounds__(WGT, 1) k_node_bwd_tc(NodeTcArgs A)
+{
+    using S = NodeSmem<SPLIT>;
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ int skip;
+    const uint32_t tmem = node_setup<SPLIT>(A, sm, A.U2h, A.U2l, A.U1h, A.U1l, skip);
+    const int f = threadIdx.x;
+    const uint32_t lane = (uint32_t)((f >> 5) * 32) << 16;
+    const uint32_t mbar = smem_u32(sm + S::MBAR);
+    uint32_t phase = 0;
+    const int64_t n_tiles = (A.N + TA - 1) / TA;
+    if (!skip) {
+        unsigned char *T = sm + S::T;
+        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+            const int64_t a0 = tile * TA;
+            tile_from<SPLIT>(T, f, a0, A.N, [&](int64_t a) { return A.Xbar[a * FF + f]; });
+            if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem, mbar, phase, A.d_err)) break;
+#pragma unroll 1
+            for (int c = 0; c < TA / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int64_t a = a0 + 32 * c + q;
+                    const float p = a < A.N ? A.P[((int64_t)A.t * A.N + a) * FF + f] : 0.0f;
+                    v[q] *= sigmoid_fast(p);
+                }
+                store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
+            }
+            if (!gemm_step<SPLIT, true>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err)) break;
+#pragma unroll 1
+            for (int c = 0; c < TA / 32; ++c) {
+                float v[32];
+                tmem_ld32(tmem + lane + 128 + 32 * c, v);
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const int64_t a = a0 + 32 * c + q;
+                    if (a < A.N) A.Hbar[a * FF + f] = v[q];
+                }
+            }
+            tc_fence_before();
+            __syncthreads();
+        }
+    }
+    node_teardown(tmem);
+}
+
+template <typename Kern>
+cudaError_t launch_k(Kern k, uint32_t bytes, int grid, const NodeTcArgs &a, cudaStream_t s)
+{
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    k<<<grid, WGT, bytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// which: 0 update (block a.t), 1 readout (x^T = X[a.t]), 2 backward of block a.t's update
+cudaError_t launch_node_tc(const NodeTcArgs &a, bool split, int which, int n_sm, cudaStream_t s)
+{
+    const int64_t tiles = (a.N + TA - 1) / TA;
+    if (tiles == 0) return cudaSuccess;
+    // the fp16 plans (<= 128 KB, 256 TMEM columns) leave room for two CTAs per SM
+    const int per_sm = split ? 1 : 2;
+    const int grid = (int)(tiles < (int64_t)per_sm * n_sm ? tiles : (int64_t)per_sm * n_sm);
+    if (split) {
+        using S = NodeSmem<true>;
+        if (which == 0) return launch_k(k_node_update_tc<true>, S::BYTES_UPDATE, grid, a, s);
+        if (which == 1) return launch_k(k_node_readout_tc<true>, S::BYTES_READOUT, grid, a, s);
+        return launch_k(k_node_bwd_tc<true>, S::BYTES_UPDATE, grid, a, s);
+    }
+    using S = NodeSmem<false>;
+    if (which == 0) return launch_k(k_node_update_tc<false>, S::BYTES_UPDATE, grid, a, s);
+    if (which == 1) return launch_k(k_node_readout_tc<false>, S::BYTES_READOUT, grid, a, s);
+    return launch_k(k_node_bwd_tc<false>, S::BYTES_UPDATE, grid, a, s);
+}
+
+}  // namespace sn
