@@ -65,7 +65,8 @@ struct TcSmem {
     static constexpr uint32_t MBAR = FV + 12 * TE;      // uint64
     static constexpr uint32_t REGION = (MBAR + 8 + 127) / 128 * 128;
     static constexpr uint32_t HOLD = GROUPS + NW * REGION;
-    static constexpr uint32_t USED = HOLD + 16;
+    static constexpr uint32_t WMBAR = HOLD + 8;           // weight copies
+    static constexpr uint32_t USED = WMBAR + 8;
     // at least 116 KB so that no two CTAs share an SM
     static constexpr uint32_t BYTES = USED > 116 * 1024 ? USED : 116 * 1024;
 };
@@ -85,13 +86,6 @@ __device__ __forceinline__ int row_of_edge(const int32_t *__restrict__ row_ptr, 
     return lo;
 }
 
-template <int NW>
-__device__ __forceinline__ void copy_to_smem(unsigned char *dst, const void *src, uint32_t bytes)
-{
-    const uint4 *s = reinterpret_cast<const uint4 *>(src);
-    uint4 *d = reinterpret_cast<uint4 *>(dst);
-    for (uint32_t q = threadIdx.x; q < bytes / 16; q += WGT * NW) d[q] = __ldg(s + q);
-}
 
 __device__ __forceinline__ const float *feat_row(const EdgeTcArgs &A, int j)
 {
@@ -233,28 +227,33 @@ __device__ __forceinline__ void issue_mma4(unsigned char *sm, unsigned char *R, 
     }
 }
 
-// Kernel set-up: weights to shared memory, one mbarrier per warpgroup, TMEM for the CTA.
+// Kernel set-up: weights to shared memory by bulk copies, one mbarrier per warpgroup, TMEM
+// for the CTA.  Returns the TMEM base; skip is set when a latched condition (or a time-out
+// of the copies) means the kernel must do nothing.
 template <int KP, bool SPLIT, int NW>
 __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm, int &skip)
 {
     using S = TcSmem<KP, SPLIT, NW>;
     const int warp = threadIdx.x >> 5;
-    copy_to_smem<NW>(sm + S::W1, A.W1h, S::W1B);
-    copy_to_smem<NW>(sm + S::W2, A.W2h, S::W2B);
-    if (SPLIT) {
-        copy_to_smem<NW>(sm + S::W1 + S::W1B, A.W1l, S::W1B);
-        copy_to_smem<NW>(sm + S::W2 + S::W2B, A.W2l, S::W2B);
-    }
+    const uint32_t wmbar = smem_u32(sm + S::WMBAR);
     if (threadIdx.x == 0) {
         for (int g = 0; g < NW; ++g) mbar_init(smem_u32(sm + S::GROUPS + g * S::REGION + S::MBAR), 1);
+        mbar_init(wmbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
+        mbar_expect_tx(wmbar, S::NS * (S::W1B + S::W2B));
+        bulk_g2s(smem_u32(sm + S::W1), A.W1h, S::W1B, wmbar);
+        bulk_g2s(smem_u32(sm + S::W2), A.W2h, S::W2B, wmbar);
+        if (SPLIT) {
+            bulk_g2s(smem_u32(sm + S::W1 + S::W1B), A.W1l, S::W1B, wmbar);
+            bulk_g2s(smem_u32(sm + S::W2 + S::W2B), A.W2l, S::W2B, wmbar);
+        }
     }
     if (warp == 0) tmem_alloc(smem_u32(sm + S::HOLD), 128 * NW);
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (!wait_copies(wmbar, A.d_err)) skip = 1;
     return *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
 }
 

@@ -32,18 +32,12 @@ struct NodeSmem {
     static constexpr uint32_t W1 = W0 + NS * WB;    // second weight (hi, lo)
     static constexpr uint32_t T = W1 + NS * WB;
     static constexpr uint32_t MBAR = T + NS * TB;   // uint64
-    static constexpr uint32_t HOLD = MBAR + 8;      // TMEM address
-    static constexpr uint32_t PR = HOLD + 8;        // float[64][TA] readout products (readout only)
+    static constexpr uint32_t WMBAR = MBAR + 8;     // weight copies
+    static constexpr uint32_t HOLD = WMBAR + 8;     // TMEM address
+    static constexpr uint32_t PR = HOLD + 16;       // float[64][TA] readout products (readout only)
     static constexpr uint32_t BYTES_UPDATE = PR;
     static constexpr uint32_t BYTES_READOUT = PR + 64 * TA * 4;
 };
-
-__device__ __forceinline__ void copy_block(unsigned char *dst, const void *src, uint32_t bytes)
-{
-    const uint4 *s = reinterpret_cast<const uint4 *>(src);
-    uint4 *d = reinterpret_cast<uint4 *>(dst);
-    for (uint32_t q = threadIdx.x; q < bytes / 16; q += WGT) d[q] = __ldg(s + q);
-}
 
 // D[o][a] = sum_i W[o][i] T[a][i]  (TRANS = false)  or  D[i][a] = sum_o W[o][i] T[a][o]  (TRANS)
 template <bool SPLIT, bool TRANS>
@@ -108,22 +102,25 @@ __device__ __forceinline__ uint32_t node_setup(const NodeTcArgs &A, unsigned cha
                                                const void *w0l, const void *w1h, const void *w1l, int &skip)
 {
     using S = NodeSmem<SPLIT>;
-    copy_block(sm + S::W0, w0h, S::WB);
-    if (SPLIT) copy_block(sm + S::W0 + S::WB, w0l, S::WB);
-    if (w1h) {
-        copy_block(sm + S::W1, w1h, S::WB);
-        if (SPLIT) copy_block(sm + S::W1 + S::WB, w1l, S::WB);
-    }
+    const uint32_t wmbar = smem_u32(sm + S::WMBAR);
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(sm + S::MBAR), 1);
+        mbar_init(wmbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
+        mbar_expect_tx(wmbar, S::NS * S::WB * (w1h ? 2 : 1));
+        bulk_g2s(smem_u32(sm + S::W0), w0h, S::WB, wmbar);
+        if (SPLIT) bulk_g2s(smem_u32(sm + S::W0 + S::WB), w0l, S::WB, wmbar);
+        if (w1h) {
+            bulk_g2s(smem_u32(sm + S::W1), w1h, S::WB, wmbar);
+            if (SPLIT) bulk_g2s(smem_u32(sm + S::W1 + S::WB), w1l, S::WB, wmbar);
+        }
     }
     if ((threadIdx.x >> 5) == 0) tmem_alloc(smem_u32(sm + S::HOLD), 256);
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (!wait_copies(wmbar, A.d_err)) skip = 1;
     return *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
 }
 

@@ -65,6 +65,39 @@ static __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mbar, uint32_t
     return ok;
 }
 
+// Expect `bytes` of asynchronous copies on mbar (counts as this phase's one arrival).
+static __device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk copy global -> this CTA's shared memory (no multicast), completing on mbar.  Both
+// addresses 16-byte aligned, bytes a multiple of 16.
+static __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+
+// Bounded wait of the whole CTA for phase 0 of mbar (the weight copies); false on time-out.
+static __device__ __forceinline__ bool wait_copies(uint32_t mbar, int *d_err)
+{
+    const long long t0 = clock64();
+    int ok = 0;
+    for (;;) {
+        if (mbar_try_wait(mbar, 0)) {
+            ok = 1;
+            break;
+        }
+        if (clock64() - t0 > (1ll << 33)) break;
+    }
+    ok = __syncthreads_and(ok);
+    if (!ok && threadIdx.x == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
+    return ok != 0;
+}
+
 // This lane's 32 consecutive 32-bit TMEM columns starting at taddr (warp w reads lanes 32w..).
 static __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
 {
