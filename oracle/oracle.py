@@ -76,6 +76,13 @@ def _load(path):
                             f64, f64, C.c_int, P, P, P]
     L.sno_md_vv.restype = C.c_int
     L.sno_num_threads.restype = C.c_int
+    L.sno_philox4x32_10.argtypes = [P, P, P]
+    L.sno_philox4x32_10.restype = None
+    L.sno_langevin_noise.argtypes = [C.c_uint64, C.c_int64, C.c_int64, P]
+    L.sno_langevin_noise.restype = None
+    L.sno_md_langevin.argtypes = [P, f64, f64, P, i64, C.c_int, C.c_int, P, P, P, P, P,
+                                  f64, f64, C.c_int, f64, f64, C.c_uint64, C.c_int64, P, P]
+    L.sno_md_langevin.restype = C.c_int
     return L
 
 
@@ -176,3 +183,44 @@ def md_vv(model, weights, system, pos, vel, types, mass, dt, n_steps, forces=Non
     if st != 0:
         raise ValueError(f"oracle MD failed: status {st}")
     return pos, vel, forces, epot[:n_steps], ekin[:n_steps], int(ne[0])
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32-10 of a 4-word counter and 2-word key (uint32 words)."""
+    c = np.ascontiguousarray(ctr, dtype=np.uint32)
+    k = np.ascontiguousarray(key, dtype=np.uint32)
+    out = np.zeros(4, dtype=np.uint32)
+    lib().sno_philox4x32_10(_p(c), _p(k), _p(out))
+    return out
+
+
+def langevin_noise(seed: int, step: int, atom: int) -> np.ndarray:
+    xi = np.zeros(3)
+    lib().sno_langevin_noise(C.c_uint64(seed), C.c_int64(step), C.c_int64(atom), _p(xi))
+    return xi
+
+
+def md_langevin(model, weights, system, pos, vel, types, mass, dt, n_steps, temperature, friction,
+                seed, step0=0, forces=None):
+    """BAOAB Langevin in double.  Returns (pos, vel, forces, epot[n][R], ekin[n][R])."""
+    N, R = system.n_atoms, system.n_replicas
+    pos = np.array(pos, dtype=np.float64, copy=True)
+    vel = np.array(vel, dtype=np.float64, copy=True)
+    if forces is None:
+        rp, cl = neighbors(system, model.r_cut, pos.astype(np.float32),
+                           "cells" if system.periodic else "brute")
+        _, forces, _ = energy_forces(model, weights, system, pos, types, rp, cl, f64_pos=True)
+    forces = np.array(forces, dtype=np.float64, copy=True)
+    w = np.ascontiguousarray(weights, dtype=np.float32)
+    types = np.ascontiguousarray(types, dtype=np.int32)
+    epot = np.zeros((max(n_steps, 1), R))
+    ekin = np.zeros((max(n_steps, 1), R))
+    box = _box(system)
+    st = lib().sno_md_langevin(_p(_dims(model)), C.c_double(model.r_cut), C.c_double(model.gamma), _p(w),
+                               C.c_int64(w.size), system.n_per_replica, system.n_replicas, _p(box), _p(pos),
+                               _p(vel), _p(forces), _p(types), C.c_double(mass), C.c_double(dt), n_steps,
+                               C.c_double(temperature), C.c_double(friction), C.c_uint64(seed),
+                               C.c_int64(step0), _p(epot), _p(ekin))
+    if st != 0:
+        raise ValueError(f"oracle Langevin failed: status {st}")
+    return pos, vel, forces, epot[:n_steps], ekin[:n_steps]

@@ -607,3 +607,110 @@ int sno_num_threads(void)
     return 1;
 #endif
 }
+
+/* ------------------------------------------------------------------------------------------
+ * Langevin dynamics (FlashSchNet §5.1 "Experimental setting": Langevin dynamics at 300 K,
+ * 4 fs steps), integrated with the BAOAB splitting (Leimkuhler and Matthews, 2013):
+ *   B: v += dt/2 kappa F/m;  A: r += dt/2 v;
+ *   O: v = a v + b xi,  a = exp(-friction dt),  b = sqrt((1 - a^2) kB T kappa / m);
+ *   A: r += dt/2 v;  rebuild the list;  F = F(r);  B: v += dt/2 kappa F/m.
+ * xi for (step s, atom i) comes from Philox4x32-10 (Salmon, Moraes, Dror and Shaw, 2011) with
+ * counter (s mod 2^32, s / 2^32, i, 0) and key (seed mod 2^32, seed / 2^32): its four 32-bit
+ * words u_q = (r_q + 1/2) / 2^32 give xi_x, xi_y = sqrt(-2 ln u0) (cos, sin)(2 pi u1) and
+ * xi_z = sqrt(-2 ln u2) cos(2 pi u3) (Box-Muller).
+ * ---------------------------------------------------------------------------------------- */
+
+/* Philox4x32 with 10 rounds: each round multiplies words 0 and 2 by the two round constants
+ * (64-bit products), recombines the halves with words 1 and 3 and the key, and the key is
+ * advanced by the two Weyl constants between rounds. */
+void sno_philox4x32_10(const uint32_t *ctr, const uint32_t *key, uint32_t *out)
+{
+    uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint64_t p0 = (uint64_t)0xD2511F53u * c0;
+        const uint64_t p1 = (uint64_t)0xCD9E8D57u * c2;
+        const uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+        const uint32_t n1 = (uint32_t)p1;
+        const uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+        const uint32_t n3 = (uint32_t)p0;
+        c0 = n0; c1 = n1; c2 = n2; c3 = n3;
+    }
+    out[0] = c0; out[1] = c1; out[2] = c2; out[3] = c3;
+}
+
+/* the three standard normal deviates of (step, atom) */
+void sno_langevin_noise(uint64_t seed, int64_t step, int64_t atom, double *xi)
+{
+    const uint32_t ctr[4] = {(uint32_t)step, (uint32_t)((uint64_t)step >> 32), (uint32_t)atom, 0u};
+    const uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t r[4];
+    sno_philox4x32_10(ctr, key, r);
+    double u[4];
+    for (int q = 0; q < 4; ++q) u[q] = ((double)r[q] + 0.5) / 4294967296.0;
+    const double rad0 = sqrt(-2.0 * log(u[0])), rad2 = sqrt(-2.0 * log(u[2]));
+    xi[0] = rad0 * cos(2.0 * SNO_PI * u[1]);
+    xi[1] = rad0 * sin(2.0 * SNO_PI * u[1]);
+    xi[2] = rad2 * cos(2.0 * SNO_PI * u[3]);
+}
+
+int sno_md_langevin(const int32_t *dims, double r_cut, double gamma, const float *weights, int64_t n_weights,
+                    int n_per, int n_rep, const float *box, double *pos, double *vel, double *forces,
+                    const int32_t *types, double mass, double dt, int n_steps, double temperature,
+                    double friction, uint64_t seed, int64_t step0, double *epot, double *ekin)
+{
+    int64_t N = (int64_t)n_per * n_rep;
+    if (!(mass > 0) || n_steps < 0 || !(temperature >= 0) || !(friction >= 0)) return SNO_ERR_ARG;
+    int64_t cap = 64 * N + 64;
+    int32_t *row_ptr = (int32_t *)malloc(sizeof(int32_t) * (size_t)(N + 1));
+    int32_t *col = (int32_t *)malloc(sizeof(int32_t) * (size_t)cap);
+    float *pf = (float *)malloc(sizeof(float) * (size_t)(3 * N + 1));
+    double *en = (double *)malloc(sizeof(double) * (size_t)(n_rep + 1));
+    const double c = 0.5 * dt * SNO_KAPPA / mass;
+    const double kB = 0.0019872041;
+    const double a = exp(-friction * dt);
+    const double b = sqrt((1.0 - a * a) * kB * temperature * SNO_KAPPA / mass);
+    int st = SNO_OK;
+    for (int s = 0; s < n_steps && st == SNO_OK; ++s) {
+        for (int64_t i = 0; i < N; ++i) {
+            double xi[3];
+            sno_langevin_noise(seed, step0 + s, i, xi);
+            for (int d = 0; d < 3; ++d) {
+                const int64_t q = 3 * i + d;
+                vel[q] += c * forces[q];
+                pos[q] += 0.5 * dt * vel[q];
+                vel[q] = a * vel[q] + b * xi[d];
+                pos[q] += 0.5 * dt * vel[q];
+            }
+        }
+        for (int64_t q = 0; q < 3 * N; ++q) pf[q] = (float)pos[q];
+        int64_t E = 0;
+        for (;;) {
+            int periodic = box[0] > 0 && box[1] > 0 && box[2] > 0;
+            st = periodic ? sno_neighbors_cells(n_per, n_rep, box, (float)r_cut, pf, cap, row_ptr, col, &E)
+                          : sno_neighbors_brute(n_per, n_rep, box, (float)r_cut, pf, cap, row_ptr, col, &E);
+            if (st != SNO_ERR_CAPACITY) break;
+            cap = E + E / 2 + 64;
+            free(col);
+            col = (int32_t *)malloc(sizeof(int32_t) * (size_t)cap);
+        }
+        if (st) break;
+        st = sno_energy_forces_f64(dims, r_cut, gamma, weights, n_weights, n_per, n_rep, box, pos,
+                                   types, row_ptr, col, E, en, forces, NULL);
+        if (st) break;
+        for (int64_t q = 0; q < 3 * N; ++q) vel[q] += c * forces[q];
+        for (int r = 0; r < n_rep; ++r) {
+            double ke = 0.0;
+            for (int64_t q = (int64_t)r * n_per * 3; q < (int64_t)(r + 1) * n_per * 3; ++q)
+                ke += 0.5 * mass * vel[q] * vel[q] / SNO_KAPPA;
+            if (epot) epot[(int64_t)s * n_rep + r] = en[r];
+            if (ekin) ekin[(int64_t)s * n_rep + r] = ke;
+        }
+    }
+    free(row_ptr); free(col); free(pf); free(en);
+    return st;
+}

@@ -5,6 +5,7 @@ The committed oracle is never modified; each variant lives in pytest's tmp_path.
 """
 import pytest
 
+from tests import test_oracle_langevin as lv_pins
 from tests import test_oracle_md as md_pins
 from tests import test_oracle_model as model_pins
 from tests import test_oracle_neighbors as nb_pins
@@ -50,7 +51,15 @@ def _md(O):
     md_pins.test_energy_error_is_second_order(O)
 
 
-ALL = [_closed_form, _fd, _invariances, _readout, _cutoff, _neighbors, _md]
+def _langevin(O):
+    for case in [([0, 0, 0, 0], [0, 0], [0x6627E8D5, 0xE169C58D, 0xBC57AC4C, 0x9B00DBD8])]:
+        lv_pins.test_philox_known_answers(O, *case)
+    lv_pins.test_noise_is_standard_normal(O)
+    lv_pins.test_zero_friction_is_velocity_verlet(O)
+    lv_pins.test_free_particles_thermalise(O)
+
+
+ALL = [_closed_form, _fd, _invariances, _readout, _cutoff, _neighbors, _md, _langevin]
 
 # (name, original text, planted text)
 MUTATIONS = [
@@ -78,7 +87,13 @@ MUTATIONS = [
     ("min_image_sign", "dx = dx - shift;", "dx = dx + shift;"),
     ("cells_half_stencil", "for (int oz = -1; oz <= 1; ++oz)", "for (int oz = -1; oz <= 0; ++oz)"),
     ("cutoff_inclusive", "return r2 < rc2;", "return r2 <= rc2;"),
-    ("full_kick", "const double c = 0.5 * dt * SNO_KAPPA / mass;", "const double c = dt * SNO_KAPPA / mass;"),
+    ("full_kick", "const double c = 0.5 * dt * SNO_KAPPA / mass;\n    int st = SNO_OK;",
+     "const double c = dt * SNO_KAPPA / mass;\n    int st = SNO_OK;"),
+    ("philox_weyl_constant", "k1 += 0xBB67AE85u;", "k1 += 0xBB67AE84u;"),
+    ("box_muller_sin_cos", "xi[1] = rad0 * sin(2.0 * SNO_PI * u[1]);", "xi[1] = rad0 * cos(2.0 * SNO_PI * u[1]);"),
+    ("noise_same_for_all_atoms", "sno_langevin_noise(seed, step0 + s, i, xi);", "sno_langevin_noise(seed, step0 + s, 0, xi);"),
+    ("ou_variance_without_sqrt", "const double b = sqrt((1.0 - a * a) * kB * temperature * SNO_KAPPA / mass);",
+     "const double b = (1.0 - a * a) * kB * temperature * SNO_KAPPA / mass;"),
     ("drift_before_kick", "vel[q] += c * forces[q];\n            pos[q] += dt * vel[q];",
      "pos[q] += dt * vel[q];\n            vel[q] += c * forces[q];"),
 ]
