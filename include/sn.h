@@ -169,6 +169,23 @@ sn_status sn_md_step(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *v
                      int32_t n_steps, float *energy_dev, float *kinetic_dev);
 
 /*
+ * n_steps of Langevin dynamics (the integrator of FlashSchNet §5.1 "Experimental setting":
+ * Langevin dynamics at 300 K, 4 fs), BAOAB splitting, each step:
+ *   v += dt/2 kappa F/m;  r += dt/2 v;  v = a v + b xi;  r += dt/2 v;
+ *   rebuild the list;  F, E = energy_forces(r);  v += dt/2 kappa F/m,
+ * a = exp(-friction_per_fs dt), b = sqrt((1 - a^2) kB T kappa / m), kB = 0.0019872041
+ * kcal/mol/K.  xi of step s (= step0 + 0 .. n_steps-1) and atom i: Philox4x32-10 (Salmon et
+ * al., 2011) of counter (s mod 2^32, s / 2^32, i, 0) and key (seed mod 2^32, seed / 2^32); its
+ * words u_q = (r_q + 1/2) / 2^32 give xi_x, xi_y = sqrt(-2 ln u0) (cos, sin)(2 pi u1) and
+ * xi_z = sqrt(-2 ln u2) cos(2 pi u3).  Pass step0 = the number of steps already taken to
+ * continue a trajectory.  Arguments, outputs and asynchrony as for sn_md_step.
+ */
+sn_status sn_md_langevin(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *vel_dev,
+                         float *forces_dev, const int32_t *types_dev, float mass_amu, float dt_fs,
+                         int32_t n_steps, float temperature_k, float friction_per_fs, uint64_t seed,
+                         int64_t step0, float *energy_dev, float *kinetic_dev);
+
+/*
  * Same as sn_md_step with every array in host memory (pageable or pinned): copies the
  * inputs to the context's device buffers, runs the steps, copies pos, vel, forces, energy
  * and kinetic back, and synchronises.  Returns any latched device condition.

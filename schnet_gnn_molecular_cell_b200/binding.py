@@ -48,7 +48,7 @@ class TraceEntry(C.Structure):
 
 
 EXPORTS = ["sn_create", "sn_destroy", "sn_set_stream", "sn_reserve", "sn_build_neighbors",
-           "sn_energy_forces", "sn_md_step", "sn_md_step_host", "sn_sync", "sn_md_edges",
+           "sn_energy_forces", "sn_md_step", "sn_md_langevin", "sn_md_step_host", "sn_sync", "sn_md_edges",
            "sn_trace_enable", "sn_trace_read", "sn_build_neighbors_noalloc", "sn_last_error",
            "sn_version"]
 
@@ -73,6 +73,8 @@ def load():
     L.sn_energy_forces.argtypes = [P, C.POINTER(System), P, P, P, P, i64, P, P]
     L.sn_md_step.argtypes = [P, C.POINTER(System), P, P, P, P, f32, f32, i32, P, P]
     L.sn_md_step_host.argtypes = [P, C.POINTER(System), P, P, P, P, f32, f32, i32, P, P]
+    L.sn_md_langevin.argtypes = [P, C.POINTER(System), P, P, P, P, f32, f32, i32, f32, f32, C.c_uint64, i64, P, P]
+    L.sn_md_langevin.restype = C.c_int
     L.sn_sync.argtypes = [P]
     L.sn_md_edges.argtypes = [P]
     L.sn_md_edges.restype = i64
@@ -215,6 +217,19 @@ class Context:
         self._check(self._L.sn_md_step(self._h, C.byref(system_struct(system)), _ptr(pos), _ptr(vel),
                                        _ptr(forces), _ptr(types), float(mass), float(dt), int(n_steps),
                                        _ptr(energy), _ptr(kinetic)))
+
+    def md_langevin(self, system, pos, vel, forces, types, mass: float, dt: float, n_steps: int,
+                    temperature: float, friction: float, seed: int, step0: int, energy, kinetic):
+        """BAOAB Langevin steps (see sn_md_langevin); friction in 1/fs."""
+        import torch
+        for t, dtp, n in ((pos, torch.float32, "pos"), (vel, torch.float32, "vel"),
+                          (forces, torch.float32, "forces"), (types, torch.int32, "types"),
+                          (energy, torch.float32, "energy"), (kinetic, torch.float32, "kinetic")):
+            _dev_check(t, dtp, n)
+        self._check(self._L.sn_md_langevin(self._h, C.byref(system_struct(system)), _ptr(pos), _ptr(vel),
+                                           _ptr(forces), _ptr(types), float(mass), float(dt), int(n_steps),
+                                           float(temperature), float(friction), C.c_uint64(seed),
+                                           C.c_int64(step0), _ptr(energy), _ptr(kinetic)))
 
     def md_step_host(self, system, pos, vel, forces, types, mass: float, dt: float, n_steps: int,
                      energy, kinetic):

@@ -501,11 +501,21 @@ sn_status sn_energy_forces(sn_ctx *ctx, const sn_system *sys, const float *pos_d
     return enqueue_ef(ctx, sys, types_dev, row_ptr_dev, col_dev, energy_dev, forces_dev);
 }
 
-sn_status sn_md_step(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *vel_dev, float *forces_dev,
-                     const int32_t *types_dev, float mass_amu, float dt_fs, int32_t n_steps, float *energy_dev,
-                     float *kinetic_dev)
+}  // extern "C"
+
+namespace {
+
+struct LangevinParams {
+    float a, b;        // O step: v = a v + b xi
+    uint64_t seed;
+    int64_t step0;
+};
+
+// n_steps of velocity Verlet (lv == nullptr) or BAOAB Langevin, rebuilding the list every step
+sn_status md_run(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *vel_dev, float *forces_dev,
+                 const int32_t *types_dev, float mass_amu, float dt_fs, int32_t n_steps, float *energy_dev,
+                 float *kinetic_dev, const LangevinParams *lv)
 {
-    if (!ctx) return SN_ERR_INVALID_ARG;
     sn_status st;
     if ((st = check_system(ctx, sys))) return st;
     const int64_t N = n_atoms(sys);
@@ -535,8 +545,13 @@ sn_status sn_md_step(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *v
     int32_t *rp = (int32_t *)ctx->md_row_ptr.p;
     int32_t *cl = (int32_t *)ctx->md_col.p;
     for (int s = 0; s < n_steps; ++s) {
-        cudaError_t e =
-            sn::launch_kick_drift(pos_dev, vel_dev, forces_dev, 3 * N, c, dt_fs, ctx->d_err, ctx->stream, &ctx->tracer);
+        cudaError_t e;
+        if (lv)
+            e = sn::launch_langevin_baoa(pos_dev, vel_dev, forces_dev, N, c, dt_fs, lv->a, lv->b, lv->seed,
+                                         lv->step0 + s, ctx->d_err, ctx->stream, &ctx->tracer);
+        else
+            e = sn::launch_kick_drift(pos_dev, vel_dev, forces_dev, 3 * N, c, dt_fs, ctx->d_err, ctx->stream,
+                                      &ctx->tracer);
         if (e == cudaSuccess) e = sn::launch_prep_positions(pos_dev, w.pos4, N, ctx->d_err, ctx->stream, &ctx->tracer);
         if (e == cudaSuccess)
             e = sn::launch_neighbors(*sys, ctx->cfg.r_cut, w.pos4, w, rp, cl, ctx->md_cap, ctx->d_err, nullptr,
@@ -553,6 +568,38 @@ sn_status sn_md_step(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *v
                                             kinetic_dev, ctx->d_err, ctx->stream, &ctx->tracer);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "md step: replica sums");
     return SN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sn_status sn_md_step(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *vel_dev, float *forces_dev,
+                     const int32_t *types_dev, float mass_amu, float dt_fs, int32_t n_steps, float *energy_dev,
+                     float *kinetic_dev)
+{
+    if (!ctx) return SN_ERR_INVALID_ARG;
+    return md_run(ctx, sys, pos_dev, vel_dev, forces_dev, types_dev, mass_amu, dt_fs, n_steps, energy_dev,
+                  kinetic_dev, nullptr);
+}
+
+sn_status sn_md_langevin(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *vel_dev, float *forces_dev,
+                         const int32_t *types_dev, float mass_amu, float dt_fs, int32_t n_steps, float temperature_k,
+                         float friction_per_fs, uint64_t seed, int64_t step0, float *energy_dev, float *kinetic_dev)
+{
+    if (!ctx) return SN_ERR_INVALID_ARG;
+    if (!(temperature_k >= 0.0f) || isinf(temperature_k) || !(friction_per_fs >= 0.0f) || isinf(friction_per_fs) ||
+        step0 < 0 || !(mass_amu > 0.0f))
+        return fail(ctx, SN_ERR_INVALID_ARG, "bad temperature, friction, step0 or mass");
+    const double kB = 0.0019872041;   // kcal/mol/K
+    const double a = exp(-(double)friction_per_fs * (double)dt_fs);
+    LangevinParams lv;
+    lv.a = (float)a;
+    lv.b = (float)sqrt((1.0 - a * a) * kB * (double)temperature_k * (double)KAPPA / (double)mass_amu);
+    lv.seed = seed;
+    lv.step0 = step0;
+    return md_run(ctx, sys, pos_dev, vel_dev, forces_dev, types_dev, mass_amu, dt_fs, n_steps, energy_dev,
+                  kinetic_dev, &lv);
 }
 
 sn_status sn_md_step_host(sn_ctx *ctx, const sn_system *sys, float *pos_host, float *vel_host, float *forces_host,

@@ -68,9 +68,78 @@ __global__ void __launch_bounds__(RB) k_replica_sums(const float *__restrict__ e
     }
 }
 
+// Philox4x32 with 10 rounds (Salmon, Moraes, Dror and Shaw, 2011): each round multiplies
+// words 0 and 2 by the two round constants, recombines the 64-bit products with words 1 and 3
+// and the key; the key advances by the two Weyl constants between rounds.
+__device__ __forceinline__ void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uint32_t k1)
+{
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        if (r > 0) {
+            k0 += 0x9E3779B9u;
+            k1 += 0xBB67AE85u;
+        }
+        const uint32_t lo0 = 0xD2511F53u * c[0], hi0 = __umulhi(0xD2511F53u, c[0]);
+        const uint32_t lo1 = 0xCD9E8D57u * c[2], hi1 = __umulhi(0xCD9E8D57u, c[2]);
+        const uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+        c[0] = n0;
+        c[1] = lo1;
+        c[2] = n2;
+        c[3] = lo0;
+    }
+}
+
+// Three standard normal deviates of (step, atom): Philox words u_q = (r_q + 1/2) / 2^32,
+// Box-Muller (cos, sin) of (u0, u1) and cos of (u2, u3), evaluated in double.
+__device__ __forceinline__ void langevin_noise(uint64_t seed, int64_t step, int64_t atom, float (&xi)[3])
+{
+    uint32_t c[4] = {(uint32_t)step, (uint32_t)((uint64_t)step >> 32), (uint32_t)atom, 0u};
+    philox4x32_10(c, (uint32_t)seed, (uint32_t)(seed >> 32));
+    double u[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) u[q] = ((double)c[q] + 0.5) * (1.0 / 4294967296.0);
+    const double r0 = sqrt(-2.0 * log(u[0])), r2 = sqrt(-2.0 * log(u[2]));
+    double s1, c1;
+    sincospi(2.0 * u[1], &s1, &c1);
+    xi[0] = (float)(r0 * c1);
+    xi[1] = (float)(r0 * s1);
+    xi[2] = (float)(r2 * cospi(2.0 * u[3]));
+}
+
+// BAOAB first half per atom: v += c F; r += dt/2 v; v = a v + b xi; r += dt/2 v
+__global__ void k_langevin_baoa(float *__restrict__ pos, float *__restrict__ vel, const float *__restrict__ forces,
+                                int64_t N, float c, float dt, float a, float b, uint64_t seed, int64_t step,
+                                const int *__restrict__ d_err)
+{
+    if (skip_all(d_err)) return;
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= N) return;
+    float xi[3];
+    langevin_noise(seed, step, i, xi);
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+        const int64_t q = 3 * i + d;
+        float v = vel[q] + c * forces[q];
+        float x = pos[q] + 0.5f * dt * v;
+        v = a * v + b * xi[d];
+        pos[q] = x + 0.5f * dt * v;
+        vel[q] = v;
+    }
+}
+
 inline unsigned blocks_for(int64_t n, int bt) { return (unsigned)((n + bt - 1) / bt); }
 
 }  // namespace
+
+cudaError_t launch_langevin_baoa(float *pos, float *vel, const float *forces, int64_t N, float c, float dt, float a,
+                                 float b, uint64_t seed, int64_t step, int *d_err, cudaStream_t s, Tracer *tr)
+{
+    if (N == 0) return cudaSuccess;
+    trace_begin(tr, KK_KICK_DRIFT, s);
+    k_langevin_baoa<<<blocks_for(N, 128), 128, 0, s>>>(pos, vel, forces, N, c, dt, a, b, seed, step, d_err);
+    trace_end(tr, s);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t n3, float c, float dt,
                               int *d_err, cudaStream_t s, Tracer *tr)

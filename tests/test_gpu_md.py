@@ -94,3 +94,88 @@ def test_md_capacity_overflow_is_latched(dev):
     ctx.reserve(s, 4096)
     ctx.md_step(s, pos, vel, forces, types, 12.0, 2.0, 1, e, k)
     ctx.sync()
+
+
+def _zero_filter_model(n_per, n_rep, seed=9):
+    """A model whose filter output is zero, so forces vanish identically."""
+    F, K, T, nt = 128, 50, 1, 2
+    model = synth.ModelCfg(F=F, K=K, T=T, n_types=nt, r_cut=5.0)
+    blob = synth.weights_blob(F, K, T, nt, seed=3, bias_std=0.1)
+    p = nt * F + F * K + F
+    blob[p:p + F * F + F] = 0.0
+    w = synth.make_custom(model, synth.SystemCfg(n_per, n_rep), seed, "rw")
+    return model, blob, w
+
+
+@pytest.mark.parametrize("precision", [0, 1, 2])
+def test_langevin_o_step_uses_the_oracle_noise(oracle, dev, precision):
+    from schnet_gnn_molecular_cell_b200 import Context
+    model, blob, w = _zero_filter_model(64, 2)
+    s = w.system
+    ctx = Context(model, blob, precision=precision)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    v0 = np.full((128, 3), 0.02, np.float32)
+    vel = torch.from_numpy(v0.copy()).to(dev)
+    forces = torch.zeros_like(pos)
+    types = torch.from_numpy(w.types).to(dev)
+    e = torch.empty(2, device=dev)
+    k = torch.empty(2, device=dev)
+    mass, dt, temp, fr, seed, step0 = 12.0, 4.0, 300.0, 0.01, 12345, 77
+    ctx.md_langevin(s, pos, vel, forces, types, mass, dt, 1, temp, fr, seed, step0, e, k)
+    ctx.sync()
+    a = np.exp(-fr * dt)
+    b = np.sqrt((1 - a * a) * synth.KB * temp * synth.KAPPA / mass)
+    xi = np.array([oracle.langevin_noise(seed, step0, i) for i in range(128)])
+    v1 = a * v0 + b * xi
+    np.testing.assert_allclose(vel.cpu().numpy(), v1, rtol=1e-5, atol=1e-9)
+    np.testing.assert_allclose(pos.cpu().numpy(), w.pos + 0.5 * dt * (v0 + v1), rtol=1e-6, atol=1e-6)
+    assert np.all(forces.cpu().numpy() == 0.0)
+
+
+def test_langevin_matches_oracle(oracle, dev):
+    from tests.test_gpu_parity import assert_close
+    from schnet_gnn_molecular_cell_b200 import Context
+    w = synth.make_workload(1)
+    s = w.system
+    v0 = synth.maxwell_boltzmann(32, 1, 12.0, 300.0, seed=4001)
+    ctx = Context(w.model, w.weights)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.from_numpy(v0.copy()).to(dev)
+    types = torch.from_numpy(w.types).to(dev)
+    rp, cl = ctx.neighbors(s, pos)
+    _, forces = ctx.energy_forces(s, pos, types, rp, cl)
+    forces = forces.clone()
+    e = torch.empty(1, device=dev)
+    k = torch.empty(1, device=dev)
+    ctx.md_langevin(s, pos, vel, forces, types, 12.0, 4.0, 10, 300.0, 0.001, 99, 0, e, k)
+    ctx.sync()
+    p_o, v_o, f_o, epot, ekin = oracle.md_langevin(w.model, w.weights, s, w.pos, v0, w.types, 12.0, 4.0, 10,
+                                                   300.0, 0.001, seed=99)
+    p_g = pos.cpu().numpy()
+    np.testing.assert_allclose(p_g, p_o, rtol=1e-6, atol=1e-5)
+    np.testing.assert_allclose(vel.cpu().numpy(), v_o, rtol=1e-4, atol=1e-7)
+    rp, cl = oracle.neighbors(s, w.model.r_cut, p_g)
+    E_o, F_o, _ = oracle.energy_forces(w.model, w.weights, s, p_g, w.types, rp, cl)
+    assert_close(e.cpu().numpy(), E_o, "energy at final positions")
+    assert_close(forces.cpu().numpy(), F_o, "forces at final positions")
+
+
+def test_langevin_thermalises(dev):
+    from schnet_gnn_molecular_cell_b200 import Context
+    model, blob, w = _zero_filter_model(64, 4)
+    s = w.system
+    ctx = Context(model, blob, precision=1)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.full((256, 3), 0.02, device=dev)
+    forces = torch.zeros_like(pos)
+    types = torch.from_numpy(w.types).to(dev)
+    e = torch.empty(4, device=dev)
+    k = torch.empty(4, device=dev)
+    ke = []
+    for step in range(400):
+        ctx.md_langevin(s, pos, vel, forces, types, 12.0, 4.0, 1, 300.0, 0.01, 5, step, e, k)
+        if step >= 200:
+            ke.append(k.cpu().numpy().copy())
+    ctx.sync()
+    ratio = np.mean(ke) / (1.5 * 64 * synth.KB * 300.0)
+    assert abs(ratio - 1.0) < 0.05, ratio
