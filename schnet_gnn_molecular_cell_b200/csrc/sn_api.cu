@@ -385,7 +385,11 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
     m.basis.r_cut = cfg->r_cut;
     m.basis.gamma = cfg->gamma;
     m.basis.r_cut_d = (double)cfg->r_cut;
-    for (int k = 0; k < 64; ++k) m.basis.mu[k] = k < K ? (double)k * (double)cfg->r_cut / (double)(K - 1) : 0.0;
+    for (int k = 0; k < 64; ++k) {
+        m.basis.mu[k] = k < K ? (double)k * (double)cfg->r_cut / (double)(K - 1) : 0.0;
+        m.basis.mu_hi[k] = (float)m.basis.mu[k];
+        m.basis.mu_lo[k] = (float)(m.basis.mu[k] - (double)m.basis.mu_hi[k]);
+    }
     m.emb = W + o_emb;
     for (int t = 0; t < T; ++t) {
         m.blk[t].W1 = W + o_blk[t][0];

@@ -146,6 +146,7 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
         if (BWD) sPh[n] = sPxi[n] = sPhi[n] = A.emb;
     }
     const float C = 0.5f * (cospif((float)(d / A.basis.r_cut_d)) + 1.0f);
+    const float d_hi = (float)d, d_lo = (float)(d - (double)d_hi);
     unsigned char *Bh = R + S::B;
     unsigned char *Bl = Bh + S::BB;
     const uint32_t row = (uint32_t)((n & 7) * 16 + (n >> 3) * S::SW1);
@@ -158,7 +159,7 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
             const int k = 8 * q + c;
             float b = 0.0f;
             if (n < ne && k < A.basis.K) {
-                const float x = (float)(d - A.basis.mu[k]);
+                const float x = (d_hi - A.basis.mu_hi[k]) + (d_lo - A.basis.mu_lo[k]);
                 b = __expf(-A.basis.gamma * x * x) * C;
             }
             v[c] = b;
@@ -472,15 +473,16 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 const float ratio = (float)(d / A.basis.r_cut_d);
                 const float C = 0.5f * (cospif(ratio) + 1.0f);
                 const float dC = -0.5f * (float)M_PI / A.basis.r_cut * sinpif(ratio);
+                const float d_hi = (float)d, d_lo = (float)(d - (double)d_hi);
 #pragma unroll 1
-                for (int c = 0; c < KP / CH; ++c) {
-                    float gg[CH];
-                    tmem_ld<CH>(G.tm + G.lane + COL_A + CH * c, gg);
+                for (int c = 0; c < KP / 16; ++c) {
+                    float gg[16];
+                    tmem_ld<16>(G.tm + G.lane + COL_A + 16 * c, gg);
 #pragma unroll
-                    for (int q = 0; q < CH; ++q) {
-                        const int k = CH * c + q;
+                    for (int q = 0; q < 16; ++q) {
+                        const int k = 16 * c + q;
                         if (mine && k < A.basis.K) {
-                            const float x = (float)(d - A.basis.mu[k]);
+                            const float x = (d_hi - A.basis.mu_hi[k]) + (d_lo - A.basis.mu_lo[k]);
                             const float phi = __expf(-A.basis.gamma * x * x);
                             gsum = fmaf(gg[q], -2.0f * A.basis.gamma * x * phi * C + phi * dC, gsum);
                         }

@@ -88,6 +88,9 @@ struct Basis {
     float r_cut, gamma;
     double r_cut_d;
     double mu[64];
+    // mu_k = mu_hi[k] + mu_lo[k] (float pair, exact to ~2^-48 relative): d - mu_k is formed as
+    // (d_hi - mu_hi) + (d_lo - mu_lo) in float by the tensor-core kernels
+    float mu_hi[64], mu_lo[64];
 };
 
 // ---------------------------------------------------------------- neighbour list
