@@ -254,13 +254,17 @@ __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (!wait_copies(wmbar, A.d_err)) skip = 1;
     return *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
 }
 
-template <int NW>
-__device__ __forceinline__ void teardown(uint32_t tmem)
+// The weight copies land while each group gathers its first tile; a group waits for them
+// before its first MMA (wait_weights), and the CTA waits once more here so that it never
+// leaves with copies in flight (a no-op when they have landed).
+template <int KP, bool SPLIT, int NW>
+__device__ __forceinline__ void teardown(unsigned char *sm, uint32_t tmem, int *d_err)
 {
+    using S = TcSmem<KP, SPLIT, NW>;
+    wait_copies(smem_u32(sm + S::WMBAR), d_err);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -291,6 +295,14 @@ __device__ __forceinline__ Group make_group(const EdgeTcArgs &A, unsigned char *
     G.i0 = A.part[p];
     G.i1 = A.part[p + 1];
     return G;
+}
+
+template <int KP, bool SPLIT, int NW>
+__device__ __forceinline__ bool wait_weights(const Group &G, unsigned char *sm, int *d_err)
+{
+    using S = TcSmem<KP, SPLIT, NW>;
+    uint32_t parity = 0;
+    return wait_mma(G.g, smem_u32(sm + S::WMBAR), parity, d_err);
 }
 
 // Make this group's shared-memory writes visible to the tensor core, then let thread 0 of the
@@ -345,6 +357,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
             tile_prologue<KP, SPLIT, NW, false>(A, G.R, f, G.i0, G.i1, ts, ne);
+            if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
             ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, false>(sm, G.R, G.tm + COL_W); })))
@@ -381,7 +394,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
                 if (__ldg(A.row_ptr + r) == __ldg(A.row_ptr + r + 1)) A.H[(int64_t)r * FF + f] = 0.0f;
         }
     }
-    teardown<NW>(tmem0);
+    teardown<KP, SPLIT, NW>(sm, tmem0, A.d_err);
 }
 
 // Backward of one interaction block over the group's rows (see sn_ef_fp32.cu for the algebra):
@@ -417,6 +430,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
             tile_prologue<KP, SPLIT, NW, true>(A, G.R, f, G.i0, G.i1, ts, ne);
+            if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
             ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, false>(sm, G.R, G.tm + COL_W); })))
@@ -513,7 +527,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         }
         if (ok && cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
     }
-    teardown<NW>(tmem0);
+    teardown<KP, SPLIT, NW>(sm, tmem0, A.d_err);
 }
 
 template <typename Kern>

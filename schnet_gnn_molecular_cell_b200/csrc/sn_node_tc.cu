@@ -2,7 +2,8 @@
 // readout, and the backward of the update network (FlashSchNet §3.2 "update network with
 // residual connection", "Energy readout"; §4.4 applies W16A16 to the update and readout
 // networks as well as the filter network).  Per tile of TA = 128 atoms, with feature f =
-// TMEM lane f and atoms on the MMA N dimension:
+// TMEM lane f and atoms on the MMA N dimension; the CTA's NG = 4 warpgroups share the tile,
+// warpgroup g gathering and finishing atom columns [32g, 32g + 32):
 //   update   D_P = U1 h^T, p = D_P + c1;  D_Y = U2 ssp(p)^T, x^{t+1} = x^t + D_Y + c2
 //   readout  D_O = R1 x^T (R1 padded to 128 rows), o = D_O + e1; eps = R2 . ssp(o) + e2;
 //            obar = R2 (.) sigma(o); D_X = R1^T obar, xbar^T = D_X
@@ -22,6 +23,8 @@ namespace {
 using namespace tc;
 
 constexpr int TA = 128;          // atoms per tile (MMA N)
+constexpr int NG = 4;            // warpgroups per CTA, one 32-atom column chunk each
+constexpr int NT = WGT * NG;     // threads per CTA
 
 template <bool SPLIT>
 struct NodeSmem {
@@ -59,10 +62,16 @@ __device__ __forceinline__ void issue_gemm(unsigned char *W, unsigned char *T, u
     }
 }
 
+// The weight copies issued by node_setup land while the first tile is being gathered; the
+// first GEMM of a CTA waits for them (weights_ready tracks this).
 template <bool SPLIT, bool TRANS>
 __device__ __forceinline__ bool gemm_step(unsigned char *W, unsigned char *T, uint32_t d, uint32_t mbar,
-                                          uint32_t &phase, int *d_err)
+                                          uint32_t &phase, int *d_err, bool &weights_ready, uint32_t wmbar)
 {
+    if (!weights_ready) {
+        if (!wait_copies(wmbar, d_err)) return false;
+        weights_ready = true;
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -71,24 +80,22 @@ __device__ __forceinline__ bool gemm_step(unsigned char *W, unsigned char *T, ui
         issue_gemm<SPLIT, TRANS>(W, T, d);
         mma_commit(mbar);
     }
-    return wait_mma(0, mbar, phase, d_err);
+    return wait_mma_cta(mbar, phase, d_err);
 }
 
-// value(a) for the 128 atoms of the tile at column f, into the activation tile (zero past N)
+// value(a) for atoms [32g, 32g + 32) of the tile at column f, into the activation tile (zero
+// past N)
 template <bool SPLIT, typename Get>
-__device__ __forceinline__ void tile_from(unsigned char *T, int f, int64_t a0, int64_t N, Get get)
+__device__ __forceinline__ void tile_from(unsigned char *T, int f, int g, int64_t a0, int64_t N, Get get)
 {
     using S = NodeSmem<SPLIT>;
-#pragma unroll 1
-    for (int c = 0; c < TA / 32; ++c) {
-        float v[32];
+    float v[32];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const int64_t a = a0 + 32 * c + q;
-            v[q] = a < N ? get(a) : 0.0f;
-        }
-        store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
+    for (int q = 0; q < 32; ++q) {
+        const int64_t a = a0 + 32 * g + q;
+        v[q] = a < N ? get(a) : 0.0f;
     }
+    store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * g, v);
 }
 
 __device__ __forceinline__ const float *x_row(const NodeTcArgs &A, int t, int64_t a)
@@ -120,12 +127,12 @@ __device__ __forceinline__ uint32_t node_setup(const NodeTcArgs &A, unsigned cha
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (!wait_copies(wmbar, A.d_err)) skip = 1;
     return *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
 }
 
-__device__ __forceinline__ void node_teardown(uint32_t tmem)
+__device__ __forceinline__ void node_teardown(uint32_t tmem, bool weights_ready, uint32_t wmbar, int *d_err)
 {
+    if (!weights_ready) wait_copies(wmbar, d_err);   // never leave with copies in flight
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -134,26 +141,27 @@ __device__ __forceinline__ void node_teardown(uint32_t tmem)
 
 // p = U1 h + c1 (saved); x^{t+1} = x^t + U2 ssp(p) + c2
 template <bool SPLIT>
-__global__ void __launch_bounds__(WGT, 1) k_node_update_tc(NodeTcArgs A)
+__global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
 {
     using S = NodeSmem<SPLIT>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
     const uint32_t tmem = node_setup<SPLIT>(A, sm, A.U1h, A.U1l, A.U2h, A.U2l, skip);
-    const int f = threadIdx.x;
+    const int f = threadIdx.x % WGT, g = threadIdx.x / WGT, c = g;
     const uint32_t lane = (uint32_t)((f >> 5) * 32) << 16;
     const uint32_t mbar = smem_u32(sm + S::MBAR);
     uint32_t phase = 0;
+    bool ready = false;
+    const uint32_t wmbar = smem_u32(sm + S::WMBAR);
     const int64_t n_tiles = (A.N + TA - 1) / TA;
     if (!skip) {
         const float c1f = A.c1[f], c2f = A.c2[f];
         unsigned char *T = sm + S::T;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
-            tile_from<SPLIT>(T, f, a0, A.N, [&](int64_t a) { return A.H[a * FF + f]; });
-            if (!gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err)) break;
-#pragma unroll 1
-            for (int c = 0; c < TA / 32; ++c) {
+            tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.H[a * FF + f]; });
+            if (!gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar)) break;
+            {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
 #pragma unroll
@@ -165,9 +173,8 @@ __global__ void __launch_bounds__(WGT, 1) k_node_update_tc(NodeTcArgs A)
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
-            if (!gemm_step<SPLIT, false>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err)) break;
-#pragma unroll 1
-            for (int c = 0; c < TA / 32; ++c) {
+            if (!gemm_step<SPLIT, false>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar)) break;
+            {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
 #pragma unroll
@@ -180,22 +187,24 @@ __global__ void __launch_bounds__(WGT, 1) k_node_update_tc(NodeTcArgs A)
             __syncthreads();
         }
     }
-    node_teardown(tmem);
+    node_teardown(tmem, ready, wmbar, A.d_err);
 }
 
 // o = R1 x^T + e1; eps = R2 . ssp(o) + e2; xbar^T = R1^T (R2 (.) sigma(o)); forces = 0
 template <bool SPLIT>
-__global__ void __launch_bounds__(WGT, 1) k_node_readout_tc(NodeTcArgs A)
+__global__ void __launch_bounds__(NT, 1) k_node_readout_tc(NodeTcArgs A)
 {
     using S = NodeSmem<SPLIT>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
     const uint32_t tmem = node_setup<SPLIT>(A, sm, A.R1h, A.R1l, nullptr, nullptr, skip);
-    const int f = threadIdx.x;
+    const int f = threadIdx.x % WGT, g = threadIdx.x / WGT, c = g;
     const uint32_t lane = (uint32_t)((f >> 5) * 32) << 16;
     const uint32_t mbar = smem_u32(sm + S::MBAR);
     float *sPr = reinterpret_cast<float *>(sm + S::PR);
     uint32_t phase = 0;
+    bool ready = false;
+    const uint32_t wmbar = smem_u32(sm + S::WMBAR);
     const int64_t n_tiles = (A.N + TA - 1) / TA;
     const int H = FF / 2;
     if (!skip) {
@@ -203,10 +212,9 @@ __global__ void __launch_bounds__(WGT, 1) k_node_readout_tc(NodeTcArgs A)
         unsigned char *T = sm + S::T;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
-            tile_from<SPLIT>(T, f, a0, A.N, [&](int64_t a) { return A.X[((int64_t)(A.t) * A.N + a) * FF + f]; });
-            if (!gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err)) break;
-#pragma unroll 1
-            for (int c = 0; c < TA / 32; ++c) {
+            tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.X[((int64_t)(A.t) * A.N + a) * FF + f]; });
+            if (!gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar)) break;
+            {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
 #pragma unroll
@@ -217,20 +225,19 @@ __global__ void __launch_bounds__(WGT, 1) k_node_readout_tc(NodeTcArgs A)
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
-            if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem + 128, mbar, phase, A.d_err)) break;
-            {   // per-atom energy (fixed summation order) and zero forces
-                const int64_t a = a0 + f;
+            if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar)) break;
+            if (threadIdx.x < TA) {   // per-atom energy (fixed summation order) and zero forces
+                const int64_t a = a0 + threadIdx.x;
                 if (a < A.N) {
                     float e = e2;
-                    for (int k = 0; k < H; ++k) e += sPr[k * TA + f];
+                    for (int k = 0; k < H; ++k) e += sPr[k * TA + threadIdx.x];
                     A.eps[a] = e;
                     A.forces[a * 3] = 0.0f;
                     A.forces[a * 3 + 1] = 0.0f;
                     A.forces[a * 3 + 2] = 0.0f;
                 }
             }
-#pragma unroll 1
-            for (int c = 0; c < TA / 32; ++c) {
+            {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
 #pragma unroll
@@ -243,30 +250,31 @@ __global__ void __launch_bounds__(WGT, 1) k_node_readout_tc(NodeTcArgs A)
             __syncthreads();
         }
     }
-    node_teardown(tmem);
+    node_teardown(tmem, ready, wmbar, A.d_err);
 }
 
 // hbar = U1^T (sigma(p) (.) U2^T xbar)   (block t's update network, p = P[t])
 template <bool SPLIT>
-__global__ void __launch_bounds__(WGT, 1) k_node_bwd_tc(NodeTcArgs A)
+__global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
 {
     using S = NodeSmem<SPLIT>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
     const uint32_t tmem = node_setup<SPLIT>(A, sm, A.U2h, A.U2l, A.U1h, A.U1l, skip);
-    const int f = threadIdx.x;
+    const int f = threadIdx.x % WGT, g = threadIdx.x / WGT, c = g;
     const uint32_t lane = (uint32_t)((f >> 5) * 32) << 16;
     const uint32_t mbar = smem_u32(sm + S::MBAR);
     uint32_t phase = 0;
+    bool ready = false;
+    const uint32_t wmbar = smem_u32(sm + S::WMBAR);
     const int64_t n_tiles = (A.N + TA - 1) / TA;
     if (!skip) {
         unsigned char *T = sm + S::T;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
-            tile_from<SPLIT>(T, f, a0, A.N, [&](int64_t a) { return A.Xbar[a * FF + f]; });
-            if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem, mbar, phase, A.d_err)) break;
-#pragma unroll 1
-            for (int c = 0; c < TA / 32; ++c) {
+            tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.Xbar[a * FF + f]; });
+            if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar)) break;
+            {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
 #pragma unroll
@@ -277,9 +285,8 @@ __global__ void __launch_bounds__(WGT, 1) k_node_bwd_tc(NodeTcArgs A)
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
-            if (!gemm_step<SPLIT, true>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err)) break;
-#pragma unroll 1
-            for (int c = 0; c < TA / 32; ++c) {
+            if (!gemm_step<SPLIT, true>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar)) break;
+            {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
 #pragma unroll
@@ -292,7 +299,7 @@ __global__ void __launch_bounds__(WGT, 1) k_node_bwd_tc(NodeTcArgs A)
             __syncthreads();
         }
     }
-    node_teardown(tmem);
+    node_teardown(tmem, ready, wmbar, A.d_err);
 }
 
 template <typename Kern>
@@ -300,7 +307,7 @@ cudaError_t launch_k(Kern k, uint32_t bytes, int grid, const NodeTcArgs &a, cuda
 {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
-    k<<<grid, WGT, bytes, s>>>(a);
+    k<<<grid, NT, bytes, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -311,9 +318,7 @@ cudaError_t launch_node_tc(const NodeTcArgs &a, bool split, int which, int n_sm,
 {
     const int64_t tiles = (a.N + TA - 1) / TA;
     if (tiles == 0) return cudaSuccess;
-    // the fp16 plans (<= 128 KB, 256 TMEM columns) leave room for two CTAs per SM
-    const int per_sm = split ? 1 : 2;
-    const int grid = (int)(tiles < (int64_t)per_sm * n_sm ? tiles : (int64_t)per_sm * n_sm);
+    const int grid = (int)(tiles < (int64_t)n_sm ? tiles : (int64_t)n_sm);
     if (split) {
         using S = NodeSmem<true>;
         if (which == 0) return launch_k(k_node_update_tc<true>, S::BYTES_UPDATE, grid, a, s);

@@ -225,6 +225,25 @@ static __device__ __forceinline__ bool wait_mma(int g, uint32_t mbar, uint32_t &
     return ok != 0;
 }
 
+// The same wait when the whole CTA waits on one mbarrier (every thread calls it).
+static __device__ __forceinline__ bool wait_mma_cta(uint32_t mbar, uint32_t &phase, int *d_err)
+{
+    const long long t0 = clock64();
+    int ok = 0;
+    for (;;) {
+        if (mbar_try_wait(mbar, phase)) {
+            ok = 1;
+            break;
+        }
+        if (clock64() - t0 > (1ll << 33)) break;
+    }
+    phase ^= 1u;
+    ok = __syncthreads_and(ok);
+    if (!ok && threadIdx.x == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
+    tc_fence_after();
+    return ok != 0;
+}
+
 
 // Activations with the hardware exp2/log2 units (__expf, __logf): ssp(x) = max(x, 0) +
 // ln(1 + e^-|x|) - ln 2 and sigma(x) = 1 / (1 + e^-x).  Absolute error ~3e-7, below the
