@@ -66,7 +66,9 @@ struct TcSmem {
     static constexpr uint32_t REGION = (MBAR + 8 + 127) / 128 * 128;
     static constexpr uint32_t HOLD = GROUPS + NW * REGION;
     static constexpr uint32_t WMBAR = HOLD + 8;           // weight copies
-    static constexpr uint32_t USED = WMBAR + 8;
+    static constexpr uint32_t MUH = WMBAR + 8;            // float[64]: mu_k as a float pair (hi, lo)
+    static constexpr uint32_t MUL = MUH + 256;
+    static constexpr uint32_t USED = MUL + 256;
     // at least 116 KB so that no two CTAs share an SM
     static constexpr uint32_t BYTES = USED > 116 * 1024 ? USED : 116 * 1024;
 };
@@ -100,8 +102,8 @@ __device__ __forceinline__ const float *feat_row(const EdgeTcArgs &A, int j)
 // zero for k >= K and for padding edges n >= ne.  Also the feature-row pointers of source
 // and destination used by the gathers (padding edges point at row 0, never used).
 template <int KP, bool SPLIT, int NW, bool BWD>
-__device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char *R, int t, int i0, int i1, int ts,
-                                              int ne)
+__device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigned char *sm, unsigned char *R, int t,
+                                              int i0, int i1, int ts, int ne)
 {
     using S = TcSmem<KP, SPLIT, NW>;
     const int n = t & (TE - 1), half = t / TE;
@@ -145,8 +147,14 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
         sPx[n] = A.emb;
         if (BWD) sPh[n] = sPxi[n] = sPhi[n] = A.emb;
     }
+    // Padding edges (d = 0) and padding Gaussians (k >= K, mu_k = 0) get finite values that
+    // never reach a result: W1 is zero in columns k >= K, and padding edges are skipped or
+    // zeroed by every consumer.
     const float C = 0.5f * (cospif((float)(d / A.basis.r_cut_d)) + 1.0f);
     const float d_hi = (float)d, d_lo = (float)(d - (double)d_hi);
+    const float g2 = -A.basis.gamma * LOG2EF;
+    const float *mh = reinterpret_cast<const float *>(sm + S::MUH) + half * (KP / 2);
+    const float *ml = reinterpret_cast<const float *>(sm + S::MUL) + half * (KP / 2);
     unsigned char *Bh = R + S::B;
     unsigned char *Bl = Bh + S::BB;
     const uint32_t row = (uint32_t)((n & 7) * 16 + (n >> 3) * S::SW1);
@@ -156,13 +164,9 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, unsigned char
         float v[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            const int k = 8 * q + c;
-            float b = 0.0f;
-            if (n < ne && k < A.basis.K) {
-                const float x = (d_hi - A.basis.mu_hi[k]) + (d_lo - A.basis.mu_lo[k]);
-                b = __expf(-A.basis.gamma * x * x) * C;
-            }
-            v[c] = b;
+            const int k = 8 * qq + c;
+            const float x = SPLIT ? (d_hi - mh[k]) + (d_lo - ml[k]) : d_hi - mh[k];
+            v[c] = ex2_approx(x * g2 * x) * C;
         }
         store8<SPLIT>(Bh, Bl, row + (uint32_t)q * 128, v);
     }
@@ -249,6 +253,10 @@ __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm
             bulk_g2s(smem_u32(sm + S::W1 + S::W1B), A.W1l, S::W1B, wmbar);
             bulk_g2s(smem_u32(sm + S::W2 + S::W2B), A.W2l, S::W2B, wmbar);
         }
+    }
+    if (threadIdx.x < 64) {
+        reinterpret_cast<float *>(sm + S::MUH)[threadIdx.x] = A.basis.mu_hi[threadIdx.x];
+        reinterpret_cast<float *>(sm + S::MUL)[threadIdx.x] = A.basis.mu_lo[threadIdx.x];
     }
     if (warp == 0) tmem_alloc(smem_u32(sm + S::HOLD), 128 * NW);
     tc_fence_before();
@@ -356,7 +364,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
         bool ok = true;
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT, NW, false>(A, G.R, f, G.i0, G.i1, ts, ne);
+            tile_prologue<KP, SPLIT, NW, false>(A, sm, G.R, f, G.i0, G.i1, ts, ne);
             if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
             ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
@@ -429,7 +437,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         bool ok = true;
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT, NW, true>(A, G.R, f, G.i0, G.i1, ts, ne);
+            tile_prologue<KP, SPLIT, NW, true>(A, sm, G.R, f, G.i0, G.i1, ts, ne);
             if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
             ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
@@ -478,31 +486,36 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, sb);
             }
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma4<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
-            // lanes 0-15 of each warp quadrant: edge n = 16 * quadrant + lane, dbar and force
+            // D_G rows (edges) sit in lanes 0-15 of each warp's quadrant; the 16x64b loads give
+            // edge n = 16 * quadrant + 8 (l % 2) + l / 4 to lanes l and l ^ 2 of the warp, which
+            // take the even and the odd k.  dbar_n = sum_k D_G[n][k] d(bt_k)/dd and its force.
             {
-                const int l = f & 31, n = (f >> 5) * 16 + l;
-                float gsum = 0.0f;
-                const bool mine = l < 16 && n < ne;
+                const int l = f & 31, par = (l >> 1) & 1;
+                const int n = 16 * (f >> 5) + 8 * (l & 1) + (l >> 2);
+                const bool mine = n < ne;
                 const double d = mine ? sDist[n] : 0.0;
                 const float ratio = (float)(d / A.basis.r_cut_d);
                 const float C = 0.5f * (cospif(ratio) + 1.0f);
                 const float dC = -0.5f * (float)M_PI / A.basis.r_cut * sinpif(ratio);
+                const float cc = -2.0f * A.basis.gamma * C, g2 = -A.basis.gamma * LOG2EF;
                 const float d_hi = (float)d, d_lo = (float)(d - (double)d_hi);
-#pragma unroll 1
-                for (int c = 0; c < KP / 16; ++c) {
-                    float gg[16];
-                    tmem_ld<16>(G.tm + G.lane + COL_A + 16 * c, gg);
+                const float *mh = reinterpret_cast<const float *>(sm + S::MUH) + par;
+                const float *ml = reinterpret_cast<const float *>(sm + S::MUL) + par;
+                float gsum = 0.0f;
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const int k = 16 * c + q;
-                        if (mine && k < A.basis.K) {
-                            const float x = (d_hi - A.basis.mu_hi[k]) + (d_lo - A.basis.mu_lo[k]);
-                            const float phi = __expf(-A.basis.gamma * x * x);
-                            gsum = fmaf(gg[q], -2.0f * A.basis.gamma * x * phi * C + phi * dC, gsum);
-                        }
+                for (int c = 0; c < KP / 32; ++c) {
+                    float gg[16];
+                    tmem_ld16x64b_x16(G.tm + G.lane + COL_A + 32 * c, gg);
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) {
+                        const int k = 32 * c + 2 * r;   // + par
+                        const float x = SPLIT ? (d_hi - mh[k]) + (d_lo - ml[k]) : d_hi - mh[k];
+                        const float phi = ex2_approx(x * g2 * x);
+                        gsum = fmaf(gg[r], phi * fmaf(x, cc, dC), gsum);
                     }
                 }
-                if (l < 16) {
+                gsum += __shfl_xor_sync(0xffffffffu, gsum, 2);
+                if (par == 0) {
                     sFv[3 * n] = mine ? -gsum * sU[3 * n] : 0.0f;
                     sFv[3 * n + 1] = mine ? -gsum * sU[3 * n + 1] : 0.0f;
                     sFv[3 * n + 2] = mine ? -gsum * sU[3 * n + 2] : 0.0f;

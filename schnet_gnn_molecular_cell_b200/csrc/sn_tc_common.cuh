@@ -137,6 +137,23 @@ static __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[CH])
     else tmem_ld16(taddr, v);
 }
 
+// 16 lanes x 64 bits, 16 repetitions: thread t of the warp receives lane 8 (t % 2) + t / 4 of
+// the 16 lanes starting at taddr's lane, columns 2 r + (t / 2) % 2 for r = 0..15 (32 columns in
+// all), so the 16 lanes of an M = 64 accumulator quadrant are spread over all 32 threads.
+static __device__ __forceinline__ void tmem_ld16x64b_x16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x64b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // Shared-memory matrix descriptor, no swizzle (layout type 0), version 1.
 static __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
@@ -244,6 +261,16 @@ static __device__ __forceinline__ bool wait_mma_cta(uint32_t mbar, uint32_t &pha
     return ok != 0;
 }
 
+
+constexpr float LOG2EF = 1.4426950408889634f;
+
+// 2^x by the hardware exp2 unit (ex2.approx.ftz.f32, relative error ~2^-22).
+static __device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // Activations with the hardware exp2/log2 units (__expf, __logf): ssp(x) = max(x, 0) +
 // ln(1 + e^-|x|) - ln 2 and sigma(x) = 1 / (1 + e^-x).  Absolute error ~3e-7, below the
