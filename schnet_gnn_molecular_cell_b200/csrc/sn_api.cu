@@ -36,7 +36,7 @@ struct sn_ctx {
     int32_t *h_err = nullptr;          // pinned
     // workspace
     DevBuf pos4, cnt, cell_of, cell_cnt, cell_start, cell_atoms;
-    DevBuf x, p, h, hbar, xbar, eps, part;
+    DevBuf x, p, h, hbar, xbar, eps, part, dst;
     DevBuf md_row_ptr, md_col;
     int64_t md_cap = 0;                // entries of md_col
     int64_t md_last_N = 0;
@@ -201,6 +201,8 @@ sn::EfWork ef_work(sn_ctx *ctx)
     w.xbar = (float *)ctx->xbar.p;
     w.eps = (float *)ctx->eps.p;
     w.part = (int32_t *)ctx->part.p;
+    w.dst = (int32_t *)ctx->dst.p;
+    w.dst_cap = (int64_t)(ctx->dst.bytes / sizeof(int32_t));
     w.G = edge_grid(ctx);
     return w;
 }
@@ -429,7 +431,7 @@ sn_status sn_destroy(sn_ctx *ctx)
     if (!ctx) return SN_ERR_INVALID_ARG;
     cudaStreamSynchronize(ctx->stream);
     DevBuf *bufs[] = {&ctx->pos4, &ctx->cnt, &ctx->cell_of, &ctx->cell_cnt, &ctx->cell_start, &ctx->cell_atoms,
-                      &ctx->x, &ctx->p, &ctx->h, &ctx->hbar, &ctx->xbar, &ctx->eps, &ctx->part,
+                      &ctx->x, &ctx->p, &ctx->h, &ctx->hbar, &ctx->xbar, &ctx->eps, &ctx->part, &ctx->dst,
                       &ctx->md_row_ptr, &ctx->md_col, &ctx->hc_pos, &ctx->hc_vel, &ctx->hc_forces,
                       &ctx->hc_types, &ctx->hc_energy, &ctx->hc_kin};
     for (DevBuf *b : bufs) release(*b);
@@ -500,6 +502,7 @@ sn_status sn_energy_forces(sn_ctx *ctx, const sn_system *sys, const float *pos_d
         (N > 0 && (!pos_dev || !types_dev || !forces_dev)) || (n_edges > 0 && !col_dev))
         return fail(ctx, SN_ERR_INVALID_ARG, "NULL argument");
     if ((st = ensure_ef(ctx, sys))) return st;
+    if ((st = grow(ctx, ctx->dst, sizeof(int32_t) * (size_t)n_edges))) return st;
     cudaError_t e = sn::launch_prep_positions(pos_dev, (float4 *)ctx->pos4.p, N, ctx->d_err, ctx->stream, &ctx->tracer);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "prep positions");
     return enqueue_ef(ctx, sys, types_dev, row_ptr_dev, col_dev, energy_dev, forces_dev);
@@ -543,6 +546,7 @@ sn_status md_run(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *vel_d
         if ((st = grow(ctx, ctx->md_col, sizeof(int32_t) * (size_t)(E + E / 2 + 1024)))) return st;
         ctx->md_cap = (int64_t)(ctx->md_col.bytes / sizeof(int32_t));
     }
+    if ((st = grow(ctx, ctx->dst, sizeof(int32_t) * (size_t)ctx->md_cap))) return st;
     ctx->md_last_N = N;
     const float c = 0.5f * dt_fs * KAPPA / mass_amu;
     sn::NbWork w = nb_work(ctx);

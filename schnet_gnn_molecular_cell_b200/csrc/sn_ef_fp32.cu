@@ -77,6 +77,7 @@ __device__ __forceinline__ float feat(int t, const float *__restrict__ X, const 
 struct EdgeArgs {
     const float4 *pos4;
     const int32_t *types, *row_ptr, *col, *part;
+    const int32_t *dst;    // destination row of each edge (tensor-core kernels only)
     const float *emb;
     const float *X;        // [T][N][F]
     float *H;              // [N][F] (fwd out)
@@ -565,6 +566,22 @@ __global__ void k_partition(const int32_t *__restrict__ row_ptr, int64_t N, int 
     part[c] = (int32_t)lo;
 }
 
+// dst[e] = i for every edge e of row i (the tensor-core kernels read an edge's row directly),
+// one warp per row; an edge index outside the buffer latches the capacity condition instead.
+__global__ void k_row_index(const int32_t *__restrict__ row_ptr, int64_t N, int32_t *__restrict__ dst, int64_t cap,
+                            int *__restrict__ d_err)
+{
+    const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (i >= N) return;
+    const int32_t e0 = row_ptr[i], e1 = row_ptr[i + 1];
+    if (e0 < 0 || e1 > cap) {
+        if (lane == 0) atomicOr(d_err, ERRBIT_CAPACITY);
+        return;
+    }
+    for (int32_t e = e0 + lane; e < e1; e += 32) dst[e] = (int32_t)i;
+}
+
 EdgeTcArgs tc_args(const EdgeArgs &a, const BlockW &bw, int *d_err)
 {
     EdgeTcArgs t{};
@@ -573,6 +590,7 @@ EdgeTcArgs tc_args(const EdgeArgs &a, const BlockW &bw, int *d_err)
     t.row_ptr = a.row_ptr;
     t.col = a.col;
     t.part = a.part;
+    t.dst = a.dst;
     t.emb = a.emb;
     t.X = a.X;
     t.H = a.H;
@@ -619,6 +637,8 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
     trace_begin(tr, KK_PARTITION, s);
     const int parts = m.precision == SN_PREC_FP32 ? w.G : w.G * tc_groups_per_cta(m.precision == SN_PREC_TC32);
     k_partition<<<(parts + 1 + 127) / 128, 128, 0, s>>>(row_ptr, N, parts, w.part);
+    if (m.precision != SN_PREC_FP32 && N > 0)
+        k_row_index<<<(unsigned)((32 * N + 255) / 256), 256, 0, s>>>(row_ptr, N, w.dst, w.dst_cap, d_err);
     trace_end(tr, s);
 
     EdgeArgs ea{};
@@ -627,6 +647,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
     ea.row_ptr = row_ptr;
     ea.col = col;
     ea.part = w.part;
+    ea.dst = w.dst;
     ea.emb = m.emb;
     ea.X = w.x;
     ea.H = w.h;

@@ -25,6 +25,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "sn_internal.cuh"
 #include "sn_tc_common.cuh"
 
@@ -54,11 +56,9 @@ struct TcSmem {
     // offsets inside a warpgroup region
     static constexpr uint32_t B = 0;
     static constexpr uint32_t T = B + NS * BB;
-    static constexpr uint32_t PX = T + NS * TB;         // const float *[TE]: x row of the source
-    static constexpr uint32_t PH = PX + 8 * TE;         //                    hbar row of the source
-    static constexpr uint32_t PXI = PH + 8 * TE;        //                    x row of the destination
-    static constexpr uint32_t PHI = PXI + 8 * TE;       //                    hbar row of the destination
-    static constexpr uint32_t DIST = PHI + 8 * TE;      // double[TE]
+    static constexpr uint32_t XO = T + NS * TB;         // int[TE]: offset of the source's x row
+    static constexpr uint32_t HO = XO + 4 * TE;         // int[TE]: offset of the source's hbar row
+    static constexpr uint32_t DIST = HO + 4 * TE;       // double[TE]
     static constexpr uint32_t DST = DIST + 8 * TE;      // int[TE]
     static constexpr uint32_t UVEC = DST + 4 * TE;      // float[TE][3]
     static constexpr uint32_t FV = UVEC + 12 * TE;      // float[TE][3]
@@ -77,49 +77,67 @@ struct TcSmem {
 
 namespace {
 
-__device__ __forceinline__ int row_of_edge(const int32_t *__restrict__ row_ptr, int i0, int i1, int e)
+// What a tile's prologue needs of its edge, loaded one tile ahead in two steps (indices, then
+// positions and types) so that the loads overlap the previous tile's work.
+struct EdgeIdx {
+    int i, j;
+};
+struct EdgePos {
+    float4 ri, rj;
+    int tj;
+};
+
+__device__ __forceinline__ EdgeIdx load_idx(const EdgeTcArgs &A, int e, int e1)
 {
-    int lo = i0, hi = i1 - 1;
-    while (lo < hi) {
-        int mid = (lo + hi + 1) >> 1;
-        if (__ldg(row_ptr + mid) <= e) lo = mid;
-        else hi = mid - 1;
+    EdgeIdx x{0, 0};
+    if (e < e1) {
+        x.i = __ldg(A.dst + e);
+        x.j = __ldg(A.col + e);
     }
-    return lo;
+    return x;
 }
 
-
-__device__ __forceinline__ const float *feat_row(const EdgeTcArgs &A, int j)
+__device__ __forceinline__ EdgePos load_pos(const EdgeTcArgs &A, EdgeIdx x)
 {
-    // x^0 is the embedding of the type; x^t (t >= 1) lives in X[t-1]
-    if (A.t == 0) return A.emb + (int64_t)__ldg(A.types + j) * FF;
-    return A.X + ((int64_t)(A.t - 1) * A.N + j) * FF;
+    EdgePos p;
+    p.ri = __ldg(A.pos4 + x.i);
+    p.rj = __ldg(A.pos4 + x.j);
+    p.tj = A.t == 0 ? __ldg(A.types + x.j) : 0;
+    return p;
+}
+
+// Feature rows of the current block's input x^t for thread f: x^0 is the embedding of the
+// atom's type, x^t (t >= 1) lives in X[t-1].  Source rows are gathered as base + offset with
+// the offsets of a tile kept in shared memory.
+__device__ __forceinline__ const float *x_base(const EdgeTcArgs &A, int f)
+{
+    return (A.t == 0 ? A.emb : A.X + (int64_t)(A.t - 1) * A.N * FF) + f;
+}
+
+__device__ __forceinline__ const float *x_row(const EdgeTcArgs &A, const float *xbase, int r)
+{
+    return A.t == 0 ? xbase + (int64_t)__ldg(A.types + r) * FF : xbase + (int64_t)r * FF;
 }
 
 // Edge metadata and basis rows of one tile, by the 128 threads of a warpgroup: thread t
 // handles edge n = t % 64 and half of its K_P Gaussians.  u = r_i - r_j and d in double
 // (minimum image on periodic axes); bt_k = exp(-gamma (d - mu_k)^2) C(d) as fp16 (hi/lo);
-// zero for k >= K and for padding edges n >= ne.  Also the feature-row pointers of source
-// and destination used by the gathers (padding edges point at row 0, never used).
+// also the offsets of the source's feature rows used by the gathers (padding edges: 0).
 template <int KP, bool SPLIT, int NW, bool BWD>
 __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigned char *sm, unsigned char *R, int t,
-                                              int i0, int i1, int ts, int ne)
+                                              int ne, EdgeIdx x, const EdgePos &p)
 {
     using S = TcSmem<KP, SPLIT, NW>;
     const int n = t & (TE - 1), half = t / TE;
-    const float **sPx = reinterpret_cast<const float **>(R + S::PX);
-    const float **sPh = reinterpret_cast<const float **>(R + S::PH);
-    const float **sPxi = reinterpret_cast<const float **>(R + S::PXI);
-    const float **sPhi = reinterpret_cast<const float **>(R + S::PHI);
+    int *sXo = reinterpret_cast<int *>(R + S::XO);
+    int *sHo = reinterpret_cast<int *>(R + S::HO);
     int *sDst = reinterpret_cast<int *>(R + S::DST);
     double *sDist = reinterpret_cast<double *>(R + S::DIST);
     float *sU = reinterpret_cast<float *>(R + S::UVEC);
     double d = 0.0;
     if (n < ne) {
-        const int e = ts + n;
-        const int j = __ldg(A.col + e);
-        const int i = row_of_edge(A.row_ptr, i0, i1, e);
-        const float4 ri = A.pos4[i], rj = A.pos4[j];
+        const int i = x.i, j = x.j;
+        const float4 ri = p.ri, rj = p.rj;
         double dx = (double)ri.x - (double)rj.x, dy = (double)ri.y - (double)rj.y, dz = (double)ri.z - (double)rj.z;
         if (A.geo.periodic[0]) dx -= (double)A.geo.box[0] * rint(dx / (double)A.geo.box[0]);
         if (A.geo.periodic[1]) dy -= (double)A.geo.box[1] * rint(dy / (double)A.geo.box[1]);
@@ -133,19 +151,15 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
             sU[3 * n + 1] = (float)(dy * inv);
             sU[3 * n + 2] = (float)(dz * inv);
         } else {
-            sPx[n] = feat_row(A, j);
-            if (BWD) {
-                sPh[n] = A.Hbar + (int64_t)j * FF;
-                sPxi[n] = feat_row(A, i);
-                sPhi[n] = A.Hbar + (int64_t)i * FF;
-            }
+            sXo[n] = (A.t == 0 ? p.tj : j) * FF;
+            if (BWD) sHo[n] = j * FF;
         }
     } else if (half == 0) {
         sDst[n] = -1;
         sDist[n] = 0.0;
     } else {
-        sPx[n] = A.emb;
-        if (BWD) sPh[n] = sPxi[n] = sPhi[n] = A.emb;
+        sXo[n] = 0;
+        if (BWD) sHo[n] = 0;
     }
     // Padding edges (d = 0) and padding Gaussians (k >= K, mu_k = 0) get finite values that
     // never reach a result: W1 is zero in columns k >= K, and padding edges are skipped or
@@ -355,51 +369,62 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
     if (!skip && G.i0 < G.i1) {
         const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
         const float b1f = A.b1[f], b2f = A.b2[f];
-        const float *const *sPx = reinterpret_cast<const float *const *>(G.R + S::PX);
+        const float *xbase = x_base(A, f);
+        const int *sXo = reinterpret_cast<const int *>(G.R + S::XO);
         const int *sDst = reinterpret_cast<const int *>(G.R + S::DST);
         unsigned char *Th = G.R + S::T, *Tl = Th + S::TB;
         uint32_t phase = 0;
         int cur = G.i0;
         float hacc = 0.0f;
+        // h_i += x_src (.) (w + b2) over one chunk of CH edges, running sums per destination
+        // row; a row is written when the next one starts (rows in between have no edges)
+        auto chunk = [&](int c, int ne, auto full) {
+            constexpr bool FULL = decltype(full)::value;
+            float v[CH], xs[CH];
+            tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, v);
+#pragma unroll
+            for (int q = 0; q < CH; ++q) xs[q] = __ldg(xbase + sXo[CH * c + q]);
+#pragma unroll
+            for (int q = 0; q < CH; ++q) {
+                const int n = CH * c + q;
+                if (FULL || n < ne) {
+                    const int i = sDst[n];
+                    if (i != cur) {
+                        A.H[(int64_t)cur * FF + f] = hacc;
+                        for (int r = cur + 1; r < i; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
+                        hacc = 0.0f;
+                        cur = i;
+                    }
+                    hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                }
+            }
+        };
         bool ok = true;
+        const int nf = f & (TE - 1);   // this thread's edge in every tile's prologue
+        EdgeIdx nidx = load_idx(A, e0 + nf, e1);
+        EdgePos npos = load_pos(A, nidx);
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT, NW, false>(A, sm, G.R, f, G.i0, G.i1, ts, ne);
+            tile_prologue<KP, SPLIT, NW, false>(A, sm, G.R, f, ne, nidx, npos);
+            const bool more = ts + TE < e1;
+            if (more) nidx = load_idx(A, ts + TE + nf, e1);
             if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
             ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
+            if (more) npos = load_pos(A, nidx);
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, false>(sm, G.R, G.tm + COL_W); })))
                 break;
-            // h_i += x_src (.) (w + b2), running sums per destination row
 #pragma unroll 1
             for (int c = 0; c < TE / CH; ++c) {
-                if (CH * c >= ne) break;
-                float v[CH], xs[CH];
-                tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, v);
-#pragma unroll
-                for (int q = 0; q < CH; ++q) xs[q] = __ldg(sPx[CH * c + q] + f);
-#pragma unroll
-                for (int q = 0; q < CH; ++q) {
-                    const int n = CH * c + q;
-                    if (n < ne) {
-                        const int i = sDst[n];
-                        if (i != cur) {
-                            A.H[(int64_t)cur * FF + f] = hacc;
-                            hacc = 0.0f;
-                            cur = i;
-                        }
-                        hacc = fmaf(xs[q], v[q] + b2f, hacc);
-                    }
-                }
+                if (CH * c + CH <= ne) chunk(c, ne, std::true_type{});
+                else if (CH * c < ne) chunk(c, ne, std::false_type{});
             }
             tc_fence_before();
             wg_sync(G.g);
         }
         if (ok) {
             A.H[(int64_t)cur * FF + f] = hacc;
-            // rows without edges receive no message
-            for (int r = G.i0; r < G.i1; ++r)
-                if (__ldg(A.row_ptr + r) == __ldg(A.row_ptr + r + 1)) A.H[(int64_t)r * FF + f] = 0.0f;
+            for (int r = cur + 1; r < G.i1; ++r) A.H[(int64_t)r * FF + f] = 0.0f;   // trailing rows without edges
         }
     }
     teardown<KP, SPLIT, NW>(sm, tmem0, A.d_err);
@@ -422,56 +447,84 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
     if (!skip && G.i0 < G.i1) {
         const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
         const float b1f = A.b1[f], b2f = A.b2[f];
-        const float *const *sPx = reinterpret_cast<const float *const *>(G.R + S::PX);
-        const float *const *sPh = reinterpret_cast<const float *const *>(G.R + S::PH);
-        const float *const *sPxi = reinterpret_cast<const float *const *>(G.R + S::PXI);
-        const float *const *sPhi = reinterpret_cast<const float *const *>(G.R + S::PHI);
+        const float *xbase = x_base(A, f), *hbase = A.Hbar + f;
+        const int *sXo = reinterpret_cast<const int *>(G.R + S::XO);
+        const int *sHo = reinterpret_cast<const int *>(G.R + S::HO);
         const int *sDst = reinterpret_cast<const int *>(G.R + S::DST);
         const double *sDist = reinterpret_cast<const double *>(G.R + S::DIST);
         const float *sU = reinterpret_cast<const float *>(G.R + S::UVEC);
         float *sFv = reinterpret_cast<float *>(G.R + S::FV);
         unsigned char *Th = G.R + S::T, *Tl = Th + S::TB;
         uint32_t phase = 0;
-        int cur = -1;
-        float xbacc = 0.0f, xbold = 0.0f;
         bool ok = true;
+        // Destination-row state: the running xbar sum of row cur, the row's own xbar, x_i and
+        // hbar_i, and the same values of row cur + 1 read ahead (the usual next row).
+        int cur = -1, nrow = -1;
+        float xbacc = 0.0f, xbold = 0.0f, xi_c = 0.0f, hi_c = 0.0f, nxb = 0.0f, nxi = 0.0f, nhi = 0.0f;
+        auto next_row = [&](int i) {
+            if (cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
+            xbacc = 0.0f;
+            cur = i;
+            if (i == nrow) {
+                xbold = nxb;
+                xi_c = nxi;
+                hi_c = nhi;
+            } else {
+                xbold = A.Xbar[(int64_t)i * FF + f];
+                xi_c = __ldg(x_row(A, xbase, i));
+                hi_c = __ldg(hbase + (int64_t)i * FF);
+            }
+            nrow = i + 1 < A.N ? i + 1 : -1;
+            if (nrow >= 0) {   // discarded unless row i + 1 is this group's next row
+                nxb = A.Xbar[(int64_t)nrow * FF + f];
+                nxi = __ldg(x_row(A, xbase, nrow));
+                nhi = __ldg(hbase + (int64_t)nrow * FF);
+            }
+        };
+        // xbar_i += hbar_j (.) (w + b2) and the tile of wbar = x_j (.) hbar_i + x_i (.) hbar_j over
+        // one chunk of CH edges (zero for padding edges)
+        auto chunk = [&](int c, int ne, auto full) {
+            constexpr bool FULL = decltype(full)::value;
+            float w[CH], hb[CH], xj[CH];
+            tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, w);
+#pragma unroll
+            for (int q = 0; q < CH; ++q) {
+                const int n = CH * c + q;
+                hb[q] = __ldg(hbase + sHo[n]);
+                xj[q] = __ldg(xbase + sXo[n]);
+            }
+#pragma unroll
+            for (int q = 0; q < CH; ++q) {
+                const int n = CH * c + q;
+                if (FULL || n < ne) {
+                    const int i = sDst[n];
+                    if (i != cur) next_row(i);
+                    xbacc = fmaf(hb[q], w[q] + b2f, xbacc);
+                    xj[q] = xj[q] * hi_c + xi_c * hb[q];
+                } else {
+                    xj[q] = 0.0f;
+                }
+            }
+            store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, xj);
+        };
+        const int nf = f & (TE - 1);   // this thread's edge in every tile's prologue
+        EdgeIdx nidx = load_idx(A, e0 + nf, e1);
+        EdgePos npos = load_pos(A, nidx);
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT, NW, true>(A, sm, G.R, f, G.i0, G.i1, ts, ne);
+            tile_prologue<KP, SPLIT, NW, true>(A, sm, G.R, f, ne, nidx, npos);
+            const bool more = ts + TE < e1;
+            if (more) nidx = load_idx(A, ts + TE + nf, e1);
             if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
             ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
+            if (more) npos = load_pos(A, nidx);
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, false>(sm, G.R, G.tm + COL_W); })))
                 break;
-            // xbar and wbar; source and destination features of a chunk loaded up front
 #pragma unroll 1
             for (int c = 0; c < TE / CH; ++c) {
-                float w[CH], hb[CH], xj[CH], hi_[CH], xi_[CH];
-                tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, w);
-#pragma unroll
-                for (int q = 0; q < CH; ++q) {
-                    const int n = CH * c + q;
-                    hb[q] = __ldg(sPh[n] + f);
-                    xj[q] = __ldg(sPx[n] + f);
-                    hi_[q] = __ldg(sPhi[n] + f);
-                    xi_[q] = __ldg(sPxi[n] + f);
-                }
-#pragma unroll
-                for (int q = 0; q < CH; ++q) {
-                    const int n = CH * c + q;
-                    if (n < ne) {
-                        const int i = sDst[n];
-                        if (i != cur) {
-                            if (cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
-                            xbacc = 0.0f;
-                            cur = i;
-                            xbold = A.Xbar[(int64_t)i * FF + f];   // consumed at this row's flush
-                        }
-                        xbacc = fmaf(hb[q], w[q] + b2f, xbacc);
-                    }
-                    xj[q] = n < ne ? xj[q] * hi_[q] + xi_[q] * hb[q] : 0.0f;
-                }
-                store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, xj);
+                if (CH * c + CH <= ne) chunk(c, ne, std::true_type{});
+                else chunk(c, ne, std::false_type{});
             }
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, true>(sm, G.R, G.tm + COL_W); })))
                 break;

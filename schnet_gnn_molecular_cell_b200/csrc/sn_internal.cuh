@@ -125,6 +125,8 @@ struct EfWork {
     float *xbar;         // [N][F]      dE/dx of the current block (in place)
     float *eps;          // [N]         per-atom energies
     int32_t *part;       // [4 G + 1]   rows owned by each CTA (fp32) / warpgroup (tensor cores)
+    int32_t *dst;        // [dst_cap]   destination row of every edge (tensor-core kernels)
+    int64_t dst_cap;
     int G;
 };
 
@@ -146,6 +148,7 @@ cudaError_t launch_energy_forces(const Model &m, const sn_system &sys, const Geo
 struct EdgeTcArgs {
     const float4 *pos4;
     const int32_t *types, *row_ptr, *col, *part;
+    const int32_t *dst;    // [E] destination row of each edge
     const float *emb;
     const float *X;        // [T][N][F]
     float *H;              // [N][F]
