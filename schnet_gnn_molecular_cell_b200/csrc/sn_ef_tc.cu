@@ -62,7 +62,8 @@ struct TcSmem {
     static constexpr uint32_t DST = DIST + 8 * TE;      // int[TE]
     static constexpr uint32_t UVEC = DST + 4 * TE;      // float[TE][3]
     static constexpr uint32_t FV = UVEC + 12 * TE;      // float[TE][3]
-    static constexpr uint32_t MBAR = FV + 12 * TE;      // uint64
+    static constexpr uint32_t MASK = FV + 12 * TE;      // uint32[4]: row starts, empty-row flags
+    static constexpr uint32_t MBAR = MASK + 16;         // uint64
     static constexpr uint32_t REGION = (MBAR + 8 + 127) / 128 * 128;
     static constexpr uint32_t HOLD = GROUPS + NW * REGION;
     static constexpr uint32_t WMBAR = HOLD + 8;           // weight copies
@@ -84,7 +85,8 @@ struct EdgeIdx {
 };
 struct EdgePos {
     float4 ri, rj;
-    int tj;
+    int tj, rs;   // type of the source (block 0), first edge of the destination's row
+    int rsm;      // first edge of the row before the destination's (-1 for row 0)
 };
 
 __device__ __forceinline__ EdgeIdx load_idx(const EdgeTcArgs &A, int e, int e1)
@@ -103,6 +105,8 @@ __device__ __forceinline__ EdgePos load_pos(const EdgeTcArgs &A, EdgeIdx x)
     p.ri = __ldg(A.pos4 + x.i);
     p.rj = __ldg(A.pos4 + x.j);
     p.tj = A.t == 0 ? __ldg(A.types + x.j) : 0;
+    p.rs = __ldg(A.row_ptr + x.i);
+    p.rsm = x.i > 0 ? __ldg(A.row_ptr + x.i - 1) : -1;
     return p;
 }
 
@@ -119,62 +123,75 @@ __device__ __forceinline__ const float *x_row(const EdgeTcArgs &A, const float *
     return A.t == 0 ? xbase + (int64_t)__ldg(A.types + r) * FF : xbase + (int64_t)r * FF;
 }
 
-// Edge metadata and basis rows of one tile, by the 128 threads of a warpgroup: thread t
-// handles edge n = t % 64 and half of its K_P Gaussians.  u = r_i - r_j and d in double
+// Edge metadata and basis rows of one tile, by 64 PARTS threads: thread t handles edge
+// n = t % 64 and part t / 64 of its K_P Gaussians; part 0 also stores the edge's metadata and
+// part 1 its gather offsets.  u = r_i - r_j and d in double
 // (minimum image on periodic axes); bt_k = exp(-gamma (d - mu_k)^2) C(d) as fp16 (hi/lo);
 // also the offsets of the source's feature rows used by the gathers (padding edges: 0).
-template <int KP, bool SPLIT, int NW, bool BWD>
+template <class S, int KP, bool SPLIT, bool BWD, int PARTS = 2>
 __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigned char *sm, unsigned char *R, int t,
-                                              int ne, EdgeIdx x, const EdgePos &p)
+                                              int ts, int ne, EdgeIdx x, const EdgePos &p)
 {
-    using S = TcSmem<KP, SPLIT, NW>;
-    const int n = t & (TE - 1), half = t / TE;
+    const int n = t & (TE - 1), half = t / TE;   // half: the part
+    static_assert(KP % (8 * PARTS) == 0, "Gaussians split in whole 8-column groups");
     int *sXo = reinterpret_cast<int *>(R + S::XO);
     int *sHo = reinterpret_cast<int *>(R + S::HO);
     int *sDst = reinterpret_cast<int *>(R + S::DST);
     double *sDist = reinterpret_cast<double *>(R + S::DIST);
     float *sU = reinterpret_cast<float *>(R + S::UVEC);
-    double d = 0.0;
+    // (double for the fp32-accurate split mode, float for fp16 operands)
+    using real = typename std::conditional<SPLIT, double, float>::type;
+    real d = 0;
     if (n < ne) {
         const int i = x.i, j = x.j;
         const float4 ri = p.ri, rj = p.rj;
-        double dx = (double)ri.x - (double)rj.x, dy = (double)ri.y - (double)rj.y, dz = (double)ri.z - (double)rj.z;
-        if (A.geo.periodic[0]) dx -= (double)A.geo.box[0] * rint(dx / (double)A.geo.box[0]);
-        if (A.geo.periodic[1]) dy -= (double)A.geo.box[1] * rint(dy / (double)A.geo.box[1]);
-        if (A.geo.periodic[2]) dz -= (double)A.geo.box[2] * rint(dz / (double)A.geo.box[2]);
+        real dx = (real)ri.x - (real)rj.x, dy = (real)ri.y - (real)rj.y, dz = (real)ri.z - (real)rj.z;
+        if (A.geo.periodic[0]) dx -= (real)A.geo.box[0] * rint(dx / (real)A.geo.box[0]);
+        if (A.geo.periodic[1]) dy -= (real)A.geo.box[1] * rint(dy / (real)A.geo.box[1]);
+        if (A.geo.periodic[2]) dz -= (real)A.geo.box[2] * rint(dz / (real)A.geo.box[2]);
         d = sqrt(dx * dx + dy * dy + dz * dz);
         if (half == 0) {
             sDst[n] = i;
-            sDist[n] = d;
-            const double inv = 1.0 / d;
+            sDist[n] = (double)d;
+            const real inv = (real)1 / d;
             sU[3 * n] = (float)(dx * inv);
             sU[3 * n + 1] = (float)(dy * inv);
             sU[3 * n + 2] = (float)(dz * inv);
-        } else {
+        } else if (half == 1) {
             sXo[n] = (A.t == 0 ? p.tj : j) * FF;
             if (BWD) sHo[n] = j * FF;
         }
     } else if (half == 0) {
         sDst[n] = -1;
         sDist[n] = 0.0;
-    } else {
+    } else if (half == 1) {
         sXo[n] = 0;
         if (BWD) sHo[n] = 0;
+    }
+    if (half == 0) {   // warps 0 and 1: the edges that start their row, and whether a row
+                       // without edges precedes any of them, one word each
+        const bool start = n < ne && ts + n == p.rs;
+        const unsigned b = __ballot_sync(0xffffffffu, start);
+        const unsigned g = __ballot_sync(0xffffffffu, start && p.rsm == p.rs);
+        if ((t & 31) == 0) {
+            reinterpret_cast<uint32_t *>(R + S::MASK)[t >> 5] = b;
+            reinterpret_cast<uint32_t *>(R + S::MASK)[2 + (t >> 5)] = g;
+        }
     }
     // Padding edges (d = 0) and padding Gaussians (k >= K, mu_k = 0) get finite values that
     // never reach a result: W1 is zero in columns k >= K, and padding edges are skipped or
     // zeroed by every consumer.
-    const float C = 0.5f * (cospif((float)(d / A.basis.r_cut_d)) + 1.0f);
-    const float d_hi = (float)d, d_lo = (float)(d - (double)d_hi);
+    const float C = 0.5f * (cospif(SPLIT ? (float)((double)d / A.basis.r_cut_d) : (float)d / A.basis.r_cut) + 1.0f);
+    const float d_hi = (float)d, d_lo = SPLIT ? (float)((double)d - (double)d_hi) : 0.0f;
     const float g2 = -A.basis.gamma * LOG2EF;
-    const float *mh = reinterpret_cast<const float *>(sm + S::MUH) + half * (KP / 2);
-    const float *ml = reinterpret_cast<const float *>(sm + S::MUL) + half * (KP / 2);
+    const float *mh = reinterpret_cast<const float *>(sm + S::MUH) + half * (KP / PARTS);
+    const float *ml = reinterpret_cast<const float *>(sm + S::MUL) + half * (KP / PARTS);
     unsigned char *Bh = R + S::B;
     unsigned char *Bl = Bh + S::BB;
     const uint32_t row = (uint32_t)((n & 7) * 16 + (n >> 3) * S::SW1);
 #pragma unroll
-    for (int qq = 0; qq < KP / 16; ++qq) {
-        const int q = half * (KP / 16) + qq;
+    for (int qq = 0; qq < KP / (8 * PARTS); ++qq) {
+        const int q = half * (KP / (8 * PARTS)) + qq;
         float v[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -187,10 +204,9 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
 }
 
 // D_A[f][n] = sum_k W1[f][k] bt[n][k]                          (M = 128, N = TE)
-template <int KP, bool SPLIT, int NW>
+template <class S, int KP, bool SPLIT>
 __device__ __forceinline__ void issue_mma1(unsigned char *sm, unsigned char *R, uint32_t d)
 {
-    using S = TcSmem<KP, SPLIT, NW>;
     constexpr uint32_t ID = idesc_f16(128, TE, 0, 0);
     const uint32_t wh = smem_u32(sm + S::W1), wl = wh + S::W1B;
     const uint32_t bh = smem_u32(R + S::B), bl = bh + S::BB;
@@ -207,10 +223,9 @@ __device__ __forceinline__ void issue_mma1(unsigned char *sm, unsigned char *R, 
 
 // TRANS = false: D[o][n] = sum_i W2[o][i] T[n][i]   (forward filter layer 2)
 // TRANS = true : D[i][n] = sum_o W2[o][i] T[n][o]   (backward through layer 2)
-template <int KP, bool SPLIT, int NW, bool TRANS>
+template <class S, bool SPLIT, bool TRANS>
 __device__ __forceinline__ void issue_mma_w2(unsigned char *sm, unsigned char *R, uint32_t d)
 {
-    using S = TcSmem<KP, SPLIT, NW>;
     constexpr uint32_t ID = idesc_f16(128, TE, TRANS ? 1 : 0, 1);
     const uint32_t wh = smem_u32(sm + S::W2), wl = wh + S::W2B;
     const uint32_t th = smem_u32(R + S::T), tl = th + S::TB;
@@ -228,10 +243,9 @@ __device__ __forceinline__ void issue_mma_w2(unsigned char *sm, unsigned char *R
 
 // D_G[n][k] = sum_f abar[n][f] W1[f][k]   (edges on M: M = TE = 64; row n of D sits in TMEM
 // lane (n % 16) + 32 (n / 16))
-template <int KP, bool SPLIT, int NW>
+template <class S, int KP, bool SPLIT>
 __device__ __forceinline__ void issue_mma4(unsigned char *sm, unsigned char *R, uint32_t d)
 {
-    using S = TcSmem<KP, SPLIT, NW>;
     constexpr uint32_t ID = idesc_f16(TE, KP, 1, 1);
     const uint32_t wh = smem_u32(sm + S::W1), wl = wh + S::W1B;
     const uint32_t th = smem_u32(R + S::T), tl = th + S::TB;
@@ -405,14 +419,14 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
         EdgePos npos = load_pos(A, nidx);
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT, NW, false>(A, sm, G.R, f, ne, nidx, npos);
+            tile_prologue<S, KP, SPLIT, false>(A, sm, G.R, f, ts, ne, nidx, npos);
             const bool more = ts + TE < e1;
             if (more) nidx = load_idx(A, ts + TE + nf, e1);
             if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<S, KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
             ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
             if (more) npos = load_pos(A, nidx);
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, false>(sm, G.R, G.tm + COL_W); })))
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
                 break;
 #pragma unroll 1
             for (int c = 0; c < TE / CH; ++c) {
@@ -512,21 +526,21 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         EdgePos npos = load_pos(A, nidx);
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<KP, SPLIT, NW, true>(A, sm, G.R, f, ne, nidx, npos);
+            tile_prologue<S, KP, SPLIT, true>(A, sm, G.R, f, ts, ne, nidx, npos);
             const bool more = ts + TE < e1;
             if (more) nidx = load_idx(A, ts + TE + nf, e1);
             if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<S, KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
             ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
             if (more) npos = load_pos(A, nidx);
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, false>(sm, G.R, G.tm + COL_W); })))
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
                 break;
 #pragma unroll 1
             for (int c = 0; c < TE / CH; ++c) {
                 if (CH * c + CH <= ne) chunk(c, ne, std::true_type{});
                 else chunk(c, ne, std::false_type{});
             }
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<KP, SPLIT, NW, true>(sm, G.R, G.tm + COL_W); })))
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, true>(sm, G.R, G.tm + COL_W); })))
                 break;
             // abar = sbar (.) sigma(a + b1)
 #pragma unroll 1
@@ -538,7 +552,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 for (int q = 0; q < CH; ++q) sb[q] *= sigmoid_fast(a[q] + b1f);
                 store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, sb);
             }
-            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma4<KP, SPLIT, NW>(sm, G.R, G.tm + COL_A); }))) break;
+            if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma4<S, KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
             // D_G rows (edges) sit in lanes 0-15 of each warp's quadrant; the 16x64b loads give
             // edge n = 16 * quadrant + 8 (l % 2) + l / 4 to lanes l and l ^ 2 of the warp, which
             // take the even and the odd k.  dbar_n = sum_k D_G[n][k] d(bt_k)/dd and its force.
@@ -596,6 +610,325 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
     teardown<KP, SPLIT, NW>(sm, tmem0, A.d_err);
 }
 
+// ---------------------------------------------------------------- warp-specialised forward
+// One CTA per SM walks the edges of its rows through a ring of NSTG tile stages, each step on
+// its own warps, so that the basis of one tile, the MMAs of another and the activations and
+// gathers of two more run at the same time:
+//   warps 0-7   P  metadata and basis tile bt of tile k, and the source   -> full_b[s]
+//                  rows x_j copied into the stage (16-byte async copies)
+//   warp  20    M  MMA1 a = W1 bt (after full_b[s])                      -> full_a[s]
+//                  MMA2 w = W2 s  (after full_t[s]), over a's columns    -> full_w[s]
+//   warps 8-15  S  s = ssp(a + b1) from TMEM into the stage's T tile     -> full_t[s]
+//                  (two warpgroups, 32 of the tile's 64 columns each)
+//   warps 16-19 E  h_i += x_j (.) (w + b2), running sums per row         -> free[s]
+// Stage s = k % NSTG holds the tile's basis and activation tiles, its metadata, the source
+// rows x_j and 64 TMEM columns.  Each barrier of stage s completes once per tile using the stage, so tile k waits
+// for parity (k / NSTG) & 1 (and P, before refilling the stage, for the previous use's free).
+constexpr int WS_WARPS = 21;
+constexpr int WS_P = 2 * WGT, WS_S = 2 * WGT;   // producer and activation threads
+constexpr int WS_M_WARP = 20;
+constexpr int WS_THREADS = WS_WARPS * 32;
+enum WsBar { WB_FULL_B = 0, WB_FULL_A, WB_FULL_T, WB_FULL_W, WB_FREE, WB_KINDS };
+
+template <int KP, bool SPLIT, int NSTG>
+struct WsSmem {
+    static constexpr int NS = SPLIT ? 2 : 1;
+    static constexpr uint32_t W1B = FF * KP * 2;
+    static constexpr uint32_t W2B = FF * FF * 2;
+    static constexpr uint32_t BB = TE * KP * 2;
+    static constexpr uint32_t TB = TE * FF * 2;
+    static constexpr uint32_t SW1 = (KP / 8) * 128;
+    static constexpr uint32_t W1 = 0;
+    static constexpr uint32_t W2 = W1 + NS * W1B;
+    static constexpr uint32_t STAGES = W2 + NS * W2B;
+    // offsets inside a stage (names as in TcSmem, which the prologue and MMA helpers use)
+    static constexpr uint32_t B = 0;
+    static constexpr uint32_t T = B + NS * BB;
+    static constexpr uint32_t XO = T + NS * TB;
+    static constexpr uint32_t HO = XO + 4 * TE;
+    static constexpr uint32_t DST = HO + 4 * TE;
+    static constexpr uint32_t DIST = DST + 4 * TE;
+    static constexpr uint32_t UVEC = DIST + 8 * TE;
+    static constexpr uint32_t FV = UVEC + 12 * TE;
+    static constexpr uint32_t MASK = FV + 12 * TE;
+    static constexpr uint32_t XS = (MASK + 16 + 127) / 128 * 128;   // float[TE][F]: x_j rows
+    static constexpr uint32_t STG = XS + TE * FF * 4;
+    static constexpr uint32_t BARS = STAGES + NSTG * STG;          // uint64 [WB_KINDS][NSTG]
+    static constexpr uint32_t WMBAR = BARS + 8 * WB_KINDS * NSTG;  // weight copies
+    static constexpr uint32_t DRAIN = WMBAR + 8;                   // last MMAs before teardown
+    static constexpr uint32_t HOLD = DRAIN + 8;                    // TMEM address
+    static constexpr uint32_t ABORT = HOLD + 8;                    // int: a wait timed out
+    static constexpr uint32_t MUH = ABORT + 8;
+    static constexpr uint32_t MUL = MUH + 256;
+    static constexpr uint32_t BYTES = MUL + 256;
+    static constexpr uint32_t TMEM_COLS = NSTG * 64 <= 128 ? 128 : NSTG * 64 <= 256 ? 256 : 512;
+};
+
+// Bounded wait on one barrier phase by every thread of a warp.  A time-out raises the CTA's
+// abort flag, which ends every other wait of the CTA at once; the result is warp-uniform.
+static __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile int *abort, int *d_err)
+{
+    const long long t0 = clock64();
+    int ok = 1;
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort) {
+            ok = 0;
+            break;
+        }
+        if (clock64() - t0 > (1ll << 32)) {
+            *abort = 1;
+            atomicOr(d_err, ERRBIT_TIMEOUT);
+            ok = 0;
+            break;
+        }
+    }
+    return __all_sync(0xffffffffu, ok) != 0;
+}
+
+template <int KP, bool SPLIT, int NSTG, int CH>
+__global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int parts_per_cta)
+{
+    using S = WsSmem<KP, SPLIT, NSTG>;
+    extern __shared__ __align__(128) unsigned char sm[];
+    __shared__ int skip;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto bar = [&](int kind, int s) { return smem_u32(sm + S::BARS + 8 * (kind * NSTG + s)); };
+    auto stage = [&](int s) { return sm + S::STAGES + s * S::STG; };
+    volatile int *abort = reinterpret_cast<volatile int *>(sm + S::ABORT);
+    const uint32_t wmbar = smem_u32(sm + S::WMBAR), drain = smem_u32(sm + S::DRAIN);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NSTG; ++s) {
+            mbar_init(bar(WB_FULL_B, s), 2 * WS_P);   // each P thread: stores, then its copies
+            mbar_init(bar(WB_FULL_A, s), 1);
+            mbar_init(bar(WB_FULL_T, s), WS_S);
+            mbar_init(bar(WB_FULL_W, s), 1);
+            mbar_init(bar(WB_FREE, s), WGT);
+        }
+        mbar_init(wmbar, 1);
+        mbar_init(drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        *abort = 0;
+        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
+        mbar_expect_tx(wmbar, S::NS * (S::W1B + S::W2B));
+        bulk_g2s(smem_u32(sm + S::W1), A.W1h, S::W1B, wmbar);
+        bulk_g2s(smem_u32(sm + S::W2), A.W2h, S::W2B, wmbar);
+        if (SPLIT) {
+            bulk_g2s(smem_u32(sm + S::W1 + S::W1B), A.W1l, S::W1B, wmbar);
+            bulk_g2s(smem_u32(sm + S::W2 + S::W2B), A.W2l, S::W2B, wmbar);
+        }
+    }
+    if (threadIdx.x < 64) {
+        reinterpret_cast<float *>(sm + S::MUH)[threadIdx.x] = A.basis.mu_hi[threadIdx.x];
+        reinterpret_cast<float *>(sm + S::MUL)[threadIdx.x] = A.basis.mu_lo[threadIdx.x];
+    }
+    if (warp == WS_M_WARP) tmem_alloc(smem_u32(sm + S::HOLD), S::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sm + S::HOLD);
+
+    const int r0 = A.part[blockIdx.x * parts_per_cta], r1 = A.part[(blockIdx.x + 1) * parts_per_cta];
+    const int e0 = r0 < r1 ? A.row_ptr[r0] : 0, e1 = r0 < r1 ? A.row_ptr[r1] : 0;
+    const int nt = (e1 - e0 + TE - 1) / TE;
+    if (!skip && r0 < r1) {
+        if (warp < 8) {
+            // P: the prologue of tile k (edge n = t % 64, a quarter of its Gaussians per
+            // thread), with tile k + 1's indices and positions read ahead
+            const int t = threadIdx.x, nf = t & (TE - 1);
+            EdgeIdx nidx = load_idx(A, e0 + nf, e1);
+            EdgePos npos = load_pos(A, nidx);
+            const float *xbase0 = x_base(A, 0);
+            for (int k = 0; k < nt; ++k) {
+                const int s = k % NSTG, ts = e0 + k * TE, ne = min(TE, e1 - ts);
+                int okw = 1;
+                if (k >= NSTG) okw = ws_wait(bar(WB_FREE, s), ((k / NSTG) - 1) & 1, abort, A.d_err);
+                if (!named_sync_and(5, WS_P, okw)) break;   // all P warps go on or stop together
+                const EdgeIdx cidx = nidx;
+                const EdgePos cpos = npos;
+                if (k + 1 < nt) nidx = load_idx(A, ts + TE + nf, e1);
+                tile_prologue<S, KP, SPLIT, false, 4>(A, sm, stage(s), t, ts, ne, cidx, cpos);
+                fence_async_smem();
+                mbar_arrive(bar(WB_FULL_B, s));
+                named_sync(5, WS_P);   // every edge's gather offset is in shared memory
+                // source rows: warp w copies rows 8w .. 8w + 7, lane l their bytes [16 l, 16 l + 16)
+                const int *sXo = reinterpret_cast<const int *>(stage(s) + S::XO);
+                const uint32_t xs = smem_u32(stage(s) + S::XS) + 16 * (t & 31);
+#pragma unroll
+                for (int r = 8 * (t >> 5); r < 8 * (t >> 5) + 8; ++r)
+                    if (r < ne) cp_async16(xs + r * FF * 4, xbase0 + sXo[r] + 4 * (t & 31));
+                cp_async_arrive(bar(WB_FULL_B, s));
+                if (k + 1 < nt) npos = load_pos(A, nidx);
+            }
+            asm volatile("cp.async.wait_all;" ::: "memory");
+        } else if (warp == WS_M_WARP) {
+            // M: lane 0 polls the two queues and issues whichever MMA is ready: MMA1 of the next
+            // tile whose basis is in (and whose stage E has released), MMA2 of the oldest tile
+            // whose activations S has written.  Decisions are broadcast so the warp stays uniform.
+            bool ok = ws_wait(wmbar, 0, abort, A.d_err);
+            bool issued = false;
+            int k1 = 0, k2 = 0;
+            long long last = clock64();
+            while (ok && k2 < nt) {
+                int go1 = 0, go2 = 0;
+                if (lane == 0) {
+                    if (k1 < nt) {
+                        const int s = k1 % NSTG;
+                        go1 = mbar_test_wait(bar(WB_FULL_B, s), (k1 / NSTG) & 1) &&
+                              (k1 < NSTG || mbar_test_wait(bar(WB_FREE, s), ((k1 / NSTG) - 1) & 1));
+                    }
+                    if (k2 < k1) go2 = mbar_test_wait(bar(WB_FULL_T, k2 % NSTG), (k2 / NSTG) & 1);
+                }
+                go1 = __shfl_sync(0xffffffffu, go1, 0);
+                go2 = __shfl_sync(0xffffffffu, go2, 0);
+                if (go1) {
+                    const int s = k1 % NSTG;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_mma1<S, KP, SPLIT>(sm, stage(s), tmem + 64 * s);
+                        mma_commit(bar(WB_FULL_A, s));
+                    }
+                    ++k1;
+                    issued = true;
+                }
+                if (go2) {
+                    const int s2 = k2 % NSTG;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        issue_mma_w2<S, SPLIT, false>(sm, stage(s2), tmem + 64 * s2);
+                        mma_commit(bar(WB_FULL_W, s2));
+                    }
+                    ++k2;
+                }
+                __syncwarp();
+                if (go1 || go2) {
+                    last = clock64();
+                } else if (*abort) {
+                    ok = false;
+                } else if (clock64() - last > (1ll << 32)) {
+                    if (lane == 0) {
+                        *abort = 1;
+                        atomicOr(A.d_err, ERRBIT_TIMEOUT);
+                    }
+                    ok = false;
+                }
+                ok = __all_sync(0xffffffffu, ok);
+            }
+            if (issued) {   // every MMA of this CTA complete before TMEM is released
+                if (lane == 0) mma_commit(drain);
+                __syncwarp();
+                const long long t0 = clock64();
+                while (!mbar_try_wait(drain, 0))
+                    if (clock64() - t0 > (1ll << 32)) {
+                        if (lane == 0) atomicOr(A.d_err, ERRBIT_TIMEOUT);
+                        break;
+                    }
+                __syncwarp();
+            }
+        } else if (warp < 16) {
+            // S: s = ssp(a + b1) into the stage's activation tile, columns [32 sg, 32 sg + 32)
+            const int f = (threadIdx.x - WS_P) % WGT, sg = (threadIdx.x - WS_P) / WGT;
+            const float b1f = A.b1[f];
+            const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
+            for (int k = 0; k < nt; ++k) {
+                const int s = k % NSTG;
+                if (!ws_wait(bar(WB_FULL_A, s), (k / NSTG) & 1, abort, A.d_err)) break;
+                tc_fence_after();
+                unsigned char *Th = stage(s) + S::T, *Tl = Th + S::TB;
+#pragma unroll 1
+                for (int c = sg * (TE / CH / 2); c < (sg + 1) * (TE / CH / 2); ++c) {
+                    float v[CH];
+                    tmem_ld<CH>(tmem + lanes + 64 * s + CH * c, v);
+#pragma unroll
+                    for (int q = 0; q < CH; ++q) v[q] = ssp_fast(v[q] + b1f);
+                    store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, v);
+                }
+                tc_fence_before();
+                fence_async_smem();
+                mbar_arrive(bar(WB_FULL_T, s));
+            }
+        } else {
+            // E: h_i += x_src (.) (w + b2); a row is written when the next one starts (rows in
+            // between, and after the last edge, have no edges and receive zero)
+            const int f = threadIdx.x - WS_P - WS_S;
+            const float b2f = A.b2[f];
+            const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
+            int cur = r0;
+            float hacc = 0.0f;
+            bool ok = true;
+            for (int k = 0; k < nt; ++k) {
+                const int s = k % NSTG, ne = min(TE, e1 - (e0 + k * TE));
+                if (!(ok = ws_wait(bar(WB_FULL_W, s), (k / NSTG) & 1, abort, A.d_err))) break;
+                // (completed already: P's metadata and the copied source rows are in place)
+                if (!(ok = ws_wait(bar(WB_FULL_B, s), (k / NSTG) & 1, abort, A.d_err))) break;
+                tc_fence_after();
+                const float *sXs = reinterpret_cast<const float *>(stage(s) + S::XS) + f;
+                const int *sDst = reinterpret_cast<const int *>(stage(s) + S::DST);
+                const uint32_t *sMask = reinterpret_cast<const uint32_t *>(stage(s) + S::MASK);
+                const uint64_t starts = (uint64_t)sMask[0] | ((uint64_t)sMask[1] << 32);
+                // A full tile with no row without edges inside takes the branch-free path: the
+                // finished row is stored under a predicate at each row start.
+                const bool fast = ne == TE && (sMask[2] | sMask[3]) == 0;
+                auto chunk = [&](int c, auto full) {
+                    constexpr bool FAST = decltype(full)::value;
+                    float v[CH], xs[CH];
+                    int dst[CH];
+                    tmem_ld<CH>(tmem + lanes + 64 * s + CH * c, v);
+#pragma unroll
+                    for (int q = 0; q < CH; ++q) {
+                        xs[q] = sXs[(CH * c + q) * FF];
+                        dst[q] = sDst[CH * c + q];
+                    }
+                    const uint32_t m = (uint32_t)(starts >> (CH * c));
+#pragma unroll
+                    for (int q = 0; q < CH; ++q) {
+                        const int n = CH * c + q;
+                        const bool st = (m >> q) & 1u;
+                        if (FAST) {
+                            store_if(A.H + (int64_t)cur * FF + f, hacc, st);
+                            hacc = st ? 0.0f : hacc;
+                            cur = st ? dst[q] : cur;
+                            hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                        } else if (n < ne) {
+                            if (st) {   // first edge of row dst[q]; rows in between have no edges
+                                store_if(A.H + (int64_t)cur * FF + f, hacc, true);
+                                for (int r = cur + 1; r < dst[q]; ++r) store_if(A.H + (int64_t)r * FF + f, 0.0f, true);
+                                hacc = 0.0f;
+                                cur = dst[q];
+                            }
+                            hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                        }
+                    }
+                };
+                if (fast) {
+#pragma unroll 1
+                    for (int c = 0; c < TE / CH; ++c) chunk(c, std::true_type{});
+                } else {
+#pragma unroll 1
+                    for (int c = 0; c < TE / CH; ++c)
+                        if (CH * c < ne) chunk(c, std::false_type{});
+                }
+                tc_fence_before();
+                mbar_arrive(bar(WB_FREE, s));
+            }
+            if (ok) {
+                store_if(A.H + (int64_t)cur * FF + f, hacc, true);
+                for (int r = cur + 1; r < r1; ++r) store_if(A.H + (int64_t)r * FF + f, 0.0f, true);
+            }
+        }
+    }
+    wait_copies(wmbar, A.d_err);   // never leave with the weight copies in flight
+    if (*abort) {
+        // after a time-out, give source-row copies that no consumer waited for time to land
+        const long long t0 = clock64();
+        while (clock64() - t0 < (1ll << 22)) {
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == WS_M_WARP) tmem_dealloc(tmem, S::TMEM_COLS);
+}
+
 template <typename Kern>
 cudaError_t prepare(Kern k, uint32_t bytes)
 {
@@ -612,6 +945,12 @@ cudaError_t launch_t(const EdgeTcArgs &a, bool backward, int G, cudaStream_t s)
     if (backward) {
         if ((e = prepare(k_edge_bwd_tc<KP, SPLIT, NW, CH>, S::BYTES))) return e;
         k_edge_bwd_tc<KP, SPLIT, NW, CH><<<G, WGT * NW, S::BYTES, s>>>(a);
+    } else if constexpr (!SPLIT) {
+        constexpr int NSTG = 3;
+        using WS = WsSmem<KP, false, NSTG>;
+        static_assert(WS::BYTES <= 227 * 1024, "shared memory plan exceeds 227 KB");
+        if ((e = prepare(k_edge_fwd_ws<KP, false, NSTG, CH>, WS::BYTES))) return e;
+        k_edge_fwd_ws<KP, false, NSTG, CH><<<G, WS_THREADS, WS::BYTES, s>>>(a, NW);
     } else {
         if ((e = prepare(k_edge_fwd_tc<KP, SPLIT, NW, CH>, S::BYTES))) return e;
         k_edge_fwd_tc<KP, SPLIT, NW, CH><<<G, WGT * NW, S::BYTES, s>>>(a);

@@ -48,6 +48,55 @@ static __device__ __forceinline__ void mma_commit(uint32_t mbar)
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
 }
 
+// Non-blocking test of a barrier phase (never suspends the thread).
+static __device__ __forceinline__ uint32_t mbar_test_wait(uint32_t mbar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    return ok;
+}
+
+// 16-byte asynchronous copy global -> shared (both 16-byte aligned), and an arrival on mbar
+// once every earlier such copy of this thread has landed (counted in the barrier's expected
+// arrivals: .noinc).
+static __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+static __device__ __forceinline__ void cp_async_arrive(uint32_t mbar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(mbar) : "memory");
+}
+
+// Named barrier over n threads that also returns whether all of them passed a true predicate.
+static __device__ __forceinline__ int named_sync_and(int id, int n, int pred)
+{
+    int out;
+    asm volatile(
+        "{\n\t.reg .pred q, p;\n\tsetp.ne.s32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\tselp.s32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(out)
+        : "r"(pred), "r"(id), "r"(n)
+        : "memory");
+    return out;
+}
+
+static __device__ __forceinline__ void named_sync(int id, int n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+static __device__ __forceinline__ void mbar_arrive(uint32_t mbar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
+}
+
 static __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
@@ -261,6 +310,14 @@ static __device__ __forceinline__ bool wait_mma_cta(uint32_t mbar, uint32_t &pha
     return ok != 0;
 }
 
+
+// Predicated global store (no branch); all stores of a value stream go through it so that
+// they keep their program order.
+static __device__ __forceinline__ void store_if(float *p, float v, bool c)
+{
+    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q st.global.f32 [%0], %1;\n\t}" ::"l"(p), "f"(v),
+                 "r"((unsigned)c));
+}
 
 constexpr float LOG2EF = 1.4426950408889634f;
 
