@@ -1,20 +1,23 @@
 // Edge kernels on the 5th-generation tensor cores (tcgen05, accumulators in TMEM).
 //
 // The filter network of every edge tile is a dense contraction (FlashSchNet §3.3 "Mixed
-// precision and Tensor Cores", §4.4): per tile of TE = 128 edges
-//   forward   D_A[f][n] = W1[f][:] . bt[n][:]          (M = F = 128, N = 128, K = K_P)
-//             D_W[f][n] = W2[f][:] . s[n][:]           (M = 128, N = 128, K = F)
-//   backward  D_S[i][n] = W2[:][i] . wbar[n][:]        (W2^T, M = 128, N = 128, K = F)
-//             D_G[n][k] = abar[n][:] . W1[:][k]        (edges on M: M = 128, N = K_P, K = F)
+// precision and Tensor Cores", §4.4): per tile of TE = 64 edges
+//   forward   D_A[f][n] = W1[f][:] . bt[n][:]          (M = F = 128, N = 64, K = K_P)
+//             D_W[f][n] = W2[f][:] . s[n][:]           (M = 128, N = 64, K = F)
+//   backward  D_S[i][n] = W2[:][i] . wbar[n][:]        (W2^T, M = 128, N = 64, K = F)
+//             D_G[n][k] = abar[n][:] . W1[:][k]        (edges on M: M = 64, N = K_P, K = F)
 // with fp16 operands in shared memory and fp32 accumulation in TMEM (the pages' W16A16 for
 // MLPs with fp32 accumulation, §4.1).  SPLIT adds an fp32-accurate mode: every operand x is
 // split into hi = fp16(x) and lo = fp16(x - hi), and each product is accumulated as
 // hi*hi + hi*lo + lo*hi (three MMAs into the same accumulator, ~22 significant bits).
 //
-// One CTA (one warpgroup of 128 threads) per SM owns whole destination rows (as the fp32
-// kernels do) and walks their edges tile by tile.  Thread t is TMEM lane t: for the
-// feature-major accumulators it is feature f = t, for D_G it is edge n = t.  The elementwise
-// work between the MMAs (Gaussians, ssp, gathers, segment sums) runs on the CUDA cores.
+// Two kernel shapes.  k_edge_fwd_tc / k_edge_bwd_tc: NW independent warpgroups per CTA (4 for
+// fp16, 2 for the split), each owning whole destination rows and walking their edges tile by
+// tile through its MMA steps; thread t of a warpgroup is TMEM lane t, i.e. feature f = t for
+// the feature-major accumulators.  k_edge_fwd_ws (fp16 forward): one warp-specialised
+// pipeline per CTA (producer, MMA, activation and epilogue warps over a ring of tile stages).
+// The elementwise work between the MMAs (Gaussians, ssp, gathers, segment sums) runs on the
+// CUDA cores.
 //
 // Shared-memory operand layout: no swizzle, 8 x 16-byte "core matrices".  An element (r, c)
 // of a matrix whose contiguous 8-element runs go along c sits at
