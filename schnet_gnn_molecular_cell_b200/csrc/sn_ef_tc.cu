@@ -369,7 +369,7 @@ __device__ __forceinline__ void ssp_to_tile(const Group &G, float b1f, unsigned 
         float v[CH];
         tmem_ld<CH>(G.tm + G.lane + COL_A + CH * c, v);
 #pragma unroll
-        for (int q = 0; q < CH; ++q) v[q] = ssp_fast(v[q] + b1f);
+        for (int q = 0; q < CH; ++q) v[q] = ssp_mode<SPLIT>(v[q] + b1f);
         store_tile_col<SPLIT, CH>(Th, Tl, G.t, CH * c, v);
     }
 }
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, sb);
                 tmem_ld<CH>(G.tm + G.lane + COL_A + CH * c, a);
 #pragma unroll
-                for (int q = 0; q < CH; ++q) sb[q] *= sigmoid_fast(a[q] + b1f);
+                for (int q = 0; q < CH; ++q) sb[q] *= sigmoid_mode<SPLIT>(a[q] + b1f);
                 store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, sb);
             }
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma4<S, KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
@@ -842,7 +842,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                     float v[CH];
                     tmem_ld<CH>(tmem + lanes + 64 * s + CH * c, v);
 #pragma unroll
-                    for (int q = 0; q < CH; ++q) v[q] = ssp_fast(v[q] + b1f);
+                    for (int q = 0; q < CH; ++q) v[q] = ssp_mode<SPLIT>(v[q] + b1f);
                     store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, v);
                 }
                 tc_fence_before();

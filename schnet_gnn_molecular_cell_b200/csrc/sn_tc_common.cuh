@@ -335,5 +335,50 @@ static __device__ __forceinline__ float ex2_approx(float x)
 static __device__ __forceinline__ float ssp_fast(float x) { return fmaxf(x, 0.0f) + __logf(1.0f + __expf(-fabsf(x))) - LN2F; }
 static __device__ __forceinline__ float sigmoid_fast(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
+// Activations for the fp16-operand mode, whose outputs are rounded to fp16 (2^-11 relative)
+// before the next MMA: one hardware transcendental each instead of two.
+//   ssp(x) = max(x, 0) + log1p(e^-|x|) - ln 2, with log1p on [0, 1] replaced by its degree-5
+//   Chebyshev interpolant at the first-kind nodes, in monomial form (max |error| 1.1e-5);
+//   sigma(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh (tanh.approx.f32).
+constexpr float LOG1P_C0 = 1.144709767686436e-05f;
+constexpr float LOG1P_C1 = 0.9991664290428162f;
+constexpr float LOG1P_C2 = -0.4896990954875946f;
+constexpr float LOG1P_C3 = 0.2838231921195984f;
+constexpr float LOG1P_C4 = -0.1299571990966797f;
+constexpr float LOG1P_C5 = 0.029808765277266502f;
+
+static __device__ __forceinline__ float ssp16(float x)
+{
+    const float u = ex2_approx(-fabsf(x) * LOG2EF);
+    float p = fmaf(LOG1P_C5, u, LOG1P_C4);
+    p = fmaf(p, u, LOG1P_C3);
+    p = fmaf(p, u, LOG1P_C2);
+    p = fmaf(p, u, LOG1P_C1);
+    p = fmaf(p, u, LOG1P_C0 - LN2F);
+    return fmaxf(x, 0.0f) + p;
+}
+
+static __device__ __forceinline__ float tanh_approx(float x)
+{
+    float y;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+static __device__ __forceinline__ float sigmoid16(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
+
+// The activation pair of a precision mode: SPLIT (fp32-accurate) or fp16 operands.
+template <bool SPLIT>
+static __device__ __forceinline__ float ssp_mode(float x)
+{
+    return SPLIT ? ssp_fast(x) : ssp16(x);
+}
+
+template <bool SPLIT>
+static __device__ __forceinline__ float sigmoid_mode(float x)
+{
+    return SPLIT ? sigmoid_fast(x) : sigmoid16(x);
+}
+
 }  // namespace tc
 }  // namespace sn
