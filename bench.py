@@ -259,6 +259,10 @@ def run_ours(args):
         flush.fill_(float(k))
         step()
     ctx.sync()
+    # the trajectory moves the edge count; the traced pass below replays the timed steps
+    # from this same state
+    saved = (pos.clone(), vel.clone(), forces.clone())
+    E_start = ctx.md_edges()
 
     uuid = None
     try:
@@ -281,22 +285,28 @@ def run_ours(args):
     clocks = sampler.stop()
     ctx.sync()
     t_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
+    E_end = ctx.md_edges()
     # per-kernel times from the library's tracer (CUDA events around every launch) on a
-    # separate pass of the same steps, so that the events do not slow the timed region
+    # separate pass over the first steps of the same trajectory, so that the events do not
+    # slow the timed region; E per traced step for the roofline's FLOP count
     n_tr = min(args.steps, 100)
+    pos.copy_(saved[0]), vel.copy_(saved[1]), forces.copy_(saved[2])
     ctx.trace(True)
+    E_tr = 0
     for k in range(n_tr):
         flush.fill_(float(k))
         step()
+        E_tr += ctx.md_edges()
     trace = ctx.trace_read()
     ctx.trace(False)
     ctx.sync()
+    E_tr /= n_tr
     if world > 1:
         t = torch.tensor([t_ms], dtype=torch.float64, device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.barrier()
         t_ms = float(t.item())
-    E_last = ctx.md_edges()
+    E_mean = 0.5 * (E_start + E_end)
     value = world * args.steps / (t_ms / 1e3)
 
     # dominant kernel and its roofline (algorithmic filter-network FLOPs per launch / mean
@@ -306,7 +316,7 @@ def run_ours(args):
     pk, pk_kind = peaks()
     roofline = None
     if dom in ("edge_fwd", "edge_bwd"):
-        flops = 2.0 * (m.K * m.F + m.F * m.F) * E_last
+        flops = 2.0 * (m.K * m.F + m.F * m.F) * E_tr
         achieved = flops / (dom_ms / launches / 1e3) / 1e12
         src = ROOT / "schnet_gnn_molecular_cell_b200" / "csrc" / ("sn_ef_fp32.cu" if prec_code == 0 else "sn_ef_tc.cu")
         if prec_code == 0:
@@ -368,10 +378,10 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": t_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": dtype, "data": "synthetic",
             "config": {"workload": WORKLOAD, "replicas_per_gpu": R, "beads": s.n_per_replica,
-                       "edges": E_last, "precision": args.precision,
+                       "edges": {"start": E_start, "end": E_end}, "precision": args.precision,
                        "l2": "flushed between steps (256 MiB write, outside the timed events)",
                        "parallelism": f"{world} rank(s), independent replica batches, no collective"},
-            "edges_per_s": value * E_last,
+            "edges_per_s": value * E_mean,
             "md_steps_x_replicas_per_s": value * R,
             "roofline": roofline,
             "cpu_baseline": cpu,

@@ -59,53 +59,45 @@ __global__ void k_prep_positions(const float *__restrict__ pos, float4 *__restri
 }
 
 // -------------------------------------------------------------------- all pairs per replica
-// grid: (ceil(n_per / BT), n_rep); FILL = false counts, true writes sources in ascending order.
+// One warp per destination atom i: lane l tests sources j = j0 + l of i's replica, a ballot
+// gives the hits in ascending j, and FILL writes them at row_ptr[i] + (hits before it) while
+// the count pass stores their number.  FILL = false counts, true writes sources in ascending
+// order.
 template <bool FILL>
-__global__ void __launch_bounds__(BT) k_pairs(const float4 *__restrict__ pos4, int n_per, Geometry g, float rc2,
-                                              int32_t *__restrict__ cnt, const int32_t *__restrict__ row_ptr,
-                                              int32_t *__restrict__ col, int64_t cap, int64_t N,
-                                              int *__restrict__ d_err)
+__global__ void __launch_bounds__(256) k_pairs(const float4 *__restrict__ pos4, int n_per, Geometry g, float rc2,
+                                               int32_t *__restrict__ cnt, const int32_t *__restrict__ row_ptr,
+                                               int32_t *__restrict__ col, int64_t cap, int64_t N,
+                                               int *__restrict__ d_err)
 {
-    __shared__ float4 tile[BT];
-    __shared__ int skip;
-    if (threadIdx.x == 0) {
-        // decided once per CTA: the loop below has barriers that every thread must reach
-        int k = (*((volatile int *)d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) ? 1 : 0;
-        if (FILL && !k && (int64_t)row_ptr[N] > cap) {
-            k = 1;
-            atomicOr(d_err, ERRBIT_CAPACITY);
-        }
-        skip = k;
+    const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (i >= N) return;
+    // (read once per warp: every exit below is taken by the whole warp)
+    const int err = __shfl_sync(0xffffffffu, lane == 0 ? *((volatile int *)d_err) : 0, 0);
+    if (err & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) return;
+    if (FILL && (int64_t)row_ptr[N] > cap) {
+        if (lane == 0) atomicOr(d_err, ERRBIT_CAPACITY);
+        return;
     }
-    __syncthreads();
-    if (skip) return;
-    const int64_t base = (int64_t)blockIdx.y * n_per;
-    const int il = blockIdx.x * BT + threadIdx.x;
-    const bool active = il < n_per;
-    const int64_t i = base + il;
-    float4 pi = active ? pos4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-    int32_t c = 0;
-    int32_t w = (FILL && active) ? row_ptr[i] : 0;
+    const int64_t base = i / n_per * n_per;
+    const int il = (int)(i - base);
+    const float4 pi = __ldg(pos4 + i);
+    int32_t w = FILL ? row_ptr[i] : 0;
     bool degenerate = false;
-    for (int j0 = 0; j0 < n_per; j0 += BT) {
-        __syncthreads();
-        if (j0 + threadIdx.x < n_per) tile[threadIdx.x] = pos4[base + j0 + threadIdx.x];
-        __syncthreads();
-        if (!active) continue;
-        const int jn = min(BT, n_per - j0);
-        for (int q = 0; q < jn; ++q) {
-            const int jl = j0 + q;
-            if (jl == il) continue;
-            float r2 = pair_r2(pi, tile[q], g);
-            if (r2 < rc2) {
-                if (FILL) col[w++] = (int32_t)(base + jl);
-                else ++c;
-                degenerate |= (r2 == 0.0f);
-            }
+    for (int j0 = 0; j0 < n_per; j0 += 32) {
+        const int jl = j0 + lane;
+        bool hit = false;
+        if (jl < n_per && jl != il) {
+            const float r2 = pair_r2(pi, __ldg(pos4 + base + jl), g);
+            hit = r2 < rc2;
+            degenerate |= hit && r2 == 0.0f;
         }
+        const unsigned m = __ballot_sync(0xffffffffu, hit);
+        if (FILL && hit) col[w + __popc(m & ((1u << lane) - 1u))] = (int32_t)(base + jl);
+        w += __popc(m);
     }
-    if (!FILL && active) cnt[i] = c;
-    if (FILL && degenerate) atomicOr(d_err, ERRBIT_DEGENERATE);
+    if (!FILL && lane == 0) cnt[i] = w;
+    if (FILL && __any_sync(0xffffffffu, degenerate) && lane == 0) atomicOr(d_err, ERRBIT_DEGENERATE);
 }
 
 // -------------------------------------------------------------------- cell list (periodic)
@@ -211,41 +203,51 @@ __global__ void __launch_bounds__(BT) k_cell_pairs(const float4 *__restrict__ po
 // -------------------------------------------------------------------- exclusive scan
 // One CTA of 1024 threads: out[0] = 0, out[k+1] = sum_{q<=k} in[q] for k < n.  Sums above
 // INT32_MAX latch ERRBIT_CAPACITY (a list that large cannot be indexed by int32).
+// out[0] = 0, out[q + 1] = in[0] + .. + in[q] (exclusive scan into n + 1 entries), by one
+// CTA of 1024 threads over tiles of 4096 entries (4 consecutive per thread), carrying the
+// running total from tile to tile; sums beyond int32 latch the capacity condition.
 __global__ void __launch_bounds__(1024) k_scan(const int32_t *__restrict__ in, int32_t *__restrict__ out, int64_t n,
                                                int *__restrict__ d_err)
 {
     __shared__ long long warp_sums[32];
-    const int t = threadIdx.x;
-    const int64_t chunk = (n + 1023) / 1024;
-    const int64_t a = t * chunk;
-    const int64_t b = min(n, a + chunk);
-    long long s = 0;
-    for (int64_t q = a; q < b; ++q) s += in[q];
-    // block exclusive scan of s
-    long long v = s;
-    const int lane = t & 31, wid = t >> 5;
-    for (int o = 1; o < 32; o <<= 1) {
-        long long y = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += y;
-    }
-    if (lane == 31) warp_sums[wid] = v;
-    __syncthreads();
-    if (wid == 0) {
-        long long ws = warp_sums[lane];
-        for (int o = 1; o < 32; o <<= 1) {
-            long long y = __shfl_up_sync(0xffffffffu, ws, o);
-            if (lane >= o) ws += y;
-        }
-        warp_sums[lane] = ws;
-    }
-    __syncthreads();
-    long long run = v - s + (wid > 0 ? warp_sums[wid - 1] : 0);
+    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
     if (t == 0) out[0] = 0;
+    long long carry = 0;
     bool over = false;
-    for (int64_t q = a; q < b; ++q) {
-        run += in[q];
-        over |= run > 0x7fffffffLL;
-        out[q + 1] = (int32_t)(run > 0x7fffffffLL ? 0x7fffffff : run);
+    for (int64_t tile = 0; tile < n; tile += 4096) {
+        const int64_t q0 = tile + 4 * t;
+        int v[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) v[k] = q0 + k < n ? in[q0 + k] : 0;
+        const long long s = (long long)v[0] + v[1] + v[2] + v[3];
+        long long x = s;   // inclusive scan of the thread sums within the warp
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            long long ws = warp_sums[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const long long y = __shfl_up_sync(0xffffffffu, ws, o);
+                if (lane >= o) ws += y;
+            }
+            warp_sums[lane] = ws;
+        }
+        __syncthreads();
+        long long run = carry + x - s + (wid > 0 ? warp_sums[wid - 1] : 0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (q0 + k < n) {
+                run += v[k];
+                over |= run > 0x7fffffffLL;
+                out[q0 + k + 1] = (int32_t)(run > 0x7fffffffLL ? 0x7fffffff : run);
+            }
+        carry += warp_sums[31];
+        __syncthreads();   // warp_sums is rewritten by the next tile
     }
     if (over) atomicOr(d_err, ERRBIT_CAPACITY);
 }
@@ -327,9 +329,9 @@ cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *po
                                                              w.cell_atoms, w.cnt, row_ptr, col, cap, d_err);
         trace_end(tr, s);
     } else {
-        dim3 grid(blocks_for(sys.n_per_replica, BT), sys.n_replicas);
         trace_begin(tr, KK_NB_COUNT, s);
-        k_pairs<false><<<grid, BT, 0, s>>>(pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col, cap, N, d_err);
+        k_pairs<false><<<blocks_for(32 * N, 256), 256, 0, s>>>(pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col,
+                                                                cap, N, d_err);
         trace_end(tr, s);
     }
     trace_begin(tr, KK_SCAN, s);
@@ -348,8 +350,8 @@ cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *po
         k_cell_pairs<true><<<blocks_for(N, BT), BT, 0, s>>>(pos4, N, g, cg, rc2, w.cell_of, w.cell_start,
                                                             w.cell_atoms, w.cnt, row_ptr, col, cap, d_err);
     } else {
-        dim3 grid(blocks_for(sys.n_per_replica, BT), sys.n_replicas);
-        k_pairs<true><<<grid, BT, 0, s>>>(pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col, cap, N, d_err);
+        k_pairs<true><<<blocks_for(32 * N, 256), 256, 0, s>>>(pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col,
+                                                               cap, N, d_err);
     }
     trace_end(tr, s);
     return cudaGetLastError();
