@@ -131,7 +131,9 @@ __device__ __forceinline__ const float *x_row(const EdgeTcArgs &A, const float *
 // part 1 its gather offsets.  u = r_i - r_j and d in double
 // (minimum image on periodic axes); bt_k = exp(-gamma (d - mu_k)^2) C(d) as fp16 (hi/lo);
 // also the offsets of the source's feature rows used by the gathers (padding edges: 0).
-template <class S, int KP, bool SPLIT, bool BWD, int PARTS = 2>
+// SHARED (fp16, warp-specialised producer): part 0 alone forms d and C(d) and leaves them in
+// the stage (S::DF, S::CC) for the other parts, after a barrier over the 64 PARTS threads.
+template <class S, int KP, bool SPLIT, bool BWD, int PARTS = 2, bool SHARED = false>
 __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigned char *sm, unsigned char *R, int t,
                                               int ts, int ne, EdgeIdx x, const EdgePos &p)
 {
@@ -145,7 +147,7 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
     // (double for the fp32-accurate split mode, float for fp16 operands)
     using real = typename std::conditional<SPLIT, double, float>::type;
     real d = 0;
-    if (n < ne) {
+    if (n < ne && (!SHARED || half <= 1)) {
         const int i = x.i, j = x.j;
         const float4 ri = p.ri, rj = p.rj;
         real dx = (real)ri.x - (real)rj.x, dy = (real)ri.y - (real)rj.y, dz = (real)ri.z - (real)rj.z;
@@ -184,8 +186,22 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
     // Padding edges (d = 0) and padding Gaussians (k >= K, mu_k = 0) get finite values that
     // never reach a result: W1 is zero in columns k >= K, and padding edges are skipped or
     // zeroed by every consumer.
-    const float C = 0.5f * (cospif(SPLIT ? (float)((double)d / A.basis.r_cut_d) : (float)d / A.basis.r_cut) + 1.0f);
-    const float d_hi = (float)d, d_lo = SPLIT ? (float)((double)d - (double)d_hi) : 0.0f;
+    float C, d_hi, d_lo;
+    if constexpr (SHARED) {
+        static_assert(!SPLIT, "shared metadata is for fp16 operands");
+        if (half == 0) {
+            reinterpret_cast<float *>(R + S::DF)[n] = (float)d;
+            reinterpret_cast<float *>(R + S::CC)[n] = 0.5f * (cospif((float)d / A.basis.r_cut) + 1.0f);
+        }
+        named_sync(5, 64 * PARTS);
+        d_hi = reinterpret_cast<const float *>(R + S::DF)[n];
+        C = reinterpret_cast<const float *>(R + S::CC)[n];
+        d_lo = 0.0f;
+    } else {
+        C = 0.5f * (cospif(SPLIT ? (float)((double)d / A.basis.r_cut_d) : (float)d / A.basis.r_cut) + 1.0f);
+        d_hi = (float)d;
+        d_lo = SPLIT ? (float)((double)d - (double)d_hi) : 0.0f;
+    }
     const float g2 = -A.basis.gamma * LOG2EF;
     const float *mh = reinterpret_cast<const float *>(sm + S::MUH) + half * (KP / PARTS);
     const float *ml = reinterpret_cast<const float *>(sm + S::MUL) + half * (KP / PARTS);
@@ -654,7 +670,9 @@ struct WsSmem {
     static constexpr uint32_t UVEC = DIST + 8 * TE;
     static constexpr uint32_t FV = UVEC + 12 * TE;
     static constexpr uint32_t MASK = FV + 12 * TE;
-    static constexpr uint32_t XS = (MASK + 16 + 127) / 128 * 128;   // float[TE][F]: x_j rows
+    static constexpr uint32_t DF = MASK + 16;                        // float[TE]: d
+    static constexpr uint32_t CC = DF + 4 * TE;                      // float[TE]: C(d)
+    static constexpr uint32_t XS = (CC + 4 * TE + 127) / 128 * 128;   // float[TE][F]: x_j rows
     static constexpr uint32_t STG = XS + TE * FF * 4;
     static constexpr uint32_t BARS = STAGES + NSTG * STG;          // uint64 [WB_KINDS][NSTG]
     static constexpr uint32_t WMBAR = BARS + 8 * WB_KINDS * NSTG;  // weight copies
@@ -749,7 +767,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                 const EdgeIdx cidx = nidx;
                 const EdgePos cpos = npos;
                 if (k + 1 < nt) nidx = load_idx(A, ts + TE + nf, e1);
-                tile_prologue<S, KP, SPLIT, false, 4>(A, sm, stage(s), t, ts, ne, cidx, cpos);
+                tile_prologue<S, KP, SPLIT, false, 4, true>(A, sm, stage(s), t, ts, ne, cidx, cpos);
                 fence_async_smem();
                 mbar_arrive(bar(WB_FULL_B, s));
                 named_sync(5, WS_P);   // every edge's gather offset is in shared memory
@@ -881,7 +899,12 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                         xs[q] = sXs[(CH * c + q) * FF];
                         dst[q] = sDst[CH * c + q];
                     }
-                    const uint32_t m = (uint32_t)(starts >> (CH * c));
+                    const uint32_t m = (uint32_t)(starts >> (CH * c)) & (CH >= 32 ? 0xffffffffu : (1u << (CH & 31)) - 1u);
+                    if (FAST && m == 0) {   // the chunk continues the current row
+#pragma unroll
+                        for (int q = 0; q < CH; ++q) hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                        return;
+                    }
 #pragma unroll
                     for (int q = 0; q < CH; ++q) {
                         const int n = CH * c + q;
