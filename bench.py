@@ -58,6 +58,9 @@ def parse():
                     help="network arithmetic: fp16 = fp16 operands on tensor cores, fp32 accumulate "
                          "(W16A16, default), tc32 = fp32-accurate fp16 split on tensor cores, fp32 = CUDA cores")
     ap.add_argument("--no-variants", action="store_true", help="skip the short runs of the other precisions")
+    ap.add_argument("--sweep", action="store_true",
+                    help="replica-scaling sweep instead of the benchmark line: one JSON line per "
+                         "(replicas, chain kind) with evals/s, steps x replicas/s and workspace bytes")
     return ap.parse_args()
 
 
@@ -398,8 +401,74 @@ def run_ours(args):
         torch.distributed.destroy_process_group()
 
 
+def run_sweep(args):
+    """Throughput against the number of replicas (1 .. 2048 chains of 269 beads) for extended
+    (self-avoiding) and compact (free random walk) chains, with the model and MD step of the
+    benchmark: the analogue of the pages' replica-scaling and dynamic-topology figures
+    (FlashSchNet §5.3).  Same timing protocol as the benchmark (CUDA events per step, L2 flushed
+    before each step); workspace = device memory the library context holds."""
+    import torch
+    from schnet_gnn_molecular_cell_b200 import Context
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    m = synth.CONFIGS[CFG]["model"]
+    w0 = synth.make_workload(CFG)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    prec_code = PRECISIONS[args.precision][0]
+    for kind in ("saw", "rw"):
+        for R in (1, 4, 16, 64, 256, 1024, 2048):
+            s = synth.SystemCfg(269, R)
+            pos0 = synth.chains(269, R, 1000 + R, saw=(kind == "saw"))
+            types = synth.bead_types(s.n_atoms, m.n_types, 2000 + R)
+            v0 = synth.maxwell_boltzmann(269, R, MASS, TEMP, 4000 + R)
+            torch.cuda.synchronize()
+            free0 = torch.cuda.mem_get_info(dev)[0]
+            ctx = Context(m, w0.weights, stream=stream, precision=prec_code)
+            pos = torch.from_numpy(pos0.copy()).to(dev)
+            vel = torch.from_numpy(v0.copy()).to(dev)
+            ty = torch.from_numpy(types).to(dev)
+            rp, cl = ctx.neighbors(s, pos)
+            E0 = int(cl.numel())
+            _, forces = ctx.energy_forces(s, pos, ty, rp, cl)
+            forces = forces.clone()
+            del rp, cl
+            ctx.reserve(s, int(1.5 * E0) + 4096)
+            e = torch.empty(R, device=dev)
+            k = torch.empty(R, device=dev)
+            steps = max(5, min(200, int(2e8 / max(E0, 1))))
+            for q in range(3):
+                flush.fill_(float(q))
+                ctx.md_step(s, pos, vel, forces, ty, MASS, DT, 1, e, k)
+            ctx.sync()
+            torch.cuda.synchronize()
+            workspace = free0 - torch.cuda.mem_get_info(dev)[0]
+            t = 0.0
+            for q in range(steps):
+                flush.fill_(float(q))
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                ctx.md_step(s, pos, vel, forces, ty, MASS, DT, 1, e, k)
+                b.record(stream)
+                b.synchronize()
+                t += a.elapsed_time(b)
+            ctx.sync()
+            E1 = ctx.md_edges()
+            ctx.close()
+            del pos, vel, ty, forces, e, k
+            rate = steps / (t / 1e3)
+            print(json.dumps({"sweep": "replicas", "kind": kind, "replicas": R, "atoms": s.n_atoms,
+                              "edges": {"start": E0, "end": E1}, "precision": args.precision, "steps": steps,
+                              "evals_per_s": rate, "md_steps_x_replicas_per_s": rate * R,
+                              "edges_per_s": rate * 0.5 * (E0 + E1), "workspace_bytes": workspace}), flush=True)
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -78,6 +78,13 @@ def test_tc32_config5(oracle, dev):
     assert_close(F_g, F_o, "forces")
 
 
+def test_fp16_config5(oracle, dev):
+    # every force component of the 65,536-atom box (2.1 M edges) in the fp16-operand mode
+    _, E_g, F_g, E_o, F_o = run(oracle, synth.make_workload(5), dev, PREC_FP16)
+    assert_close16(E_g, E_o, "energy")
+    assert_close16(F_g, F_o, "forces")
+
+
 @pytest.mark.parametrize("precision", [PREC_FP16, PREC_TC32])
 def test_tensor_modes_bitwise_deterministic_and_md(oracle, dev, precision):
     from schnet_gnn_molecular_cell_b200 import Context
