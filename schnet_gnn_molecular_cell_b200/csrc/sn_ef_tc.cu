@@ -139,8 +139,9 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
 {
     const int n = t & (TE - 1), half = t / TE;   // half: the part
     static_assert(KP % (8 * PARTS) == 0, "Gaussians split in whole 8-column groups");
+    // gather offsets: int[TE] of x rows (forward), or (x, hbar) int2[TE] over XO..HO (backward)
     int *sXo = reinterpret_cast<int *>(R + S::XO);
-    int *sHo = reinterpret_cast<int *>(R + S::HO);
+    static_assert(S::HO == S::XO + 4 * TE, "the backward's offset pairs span XO and HO");
     int *sDst = reinterpret_cast<int *>(R + S::DST);
     double *sDist = reinterpret_cast<double *>(R + S::DIST);
     float *sU = reinterpret_cast<float *>(R + S::UVEC);
@@ -163,15 +164,15 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
             sU[3 * n + 1] = (float)(dy * inv);
             sU[3 * n + 2] = (float)(dz * inv);
         } else if (half == 1) {
-            sXo[n] = (A.t == 0 ? p.tj : j) * FF;
-            if (BWD) sHo[n] = j * FF;
+            if (BWD) reinterpret_cast<int2 *>(sXo)[n] = make_int2((A.t == 0 ? p.tj : j) * FF, j * FF);
+            else sXo[n] = (A.t == 0 ? p.tj : j) * FF;
         }
     } else if (half == 0) {
         sDst[n] = -1;
         sDist[n] = 0.0;
     } else if (half == 1) {
-        sXo[n] = 0;
-        if (BWD) sHo[n] = 0;
+        if (BWD) reinterpret_cast<int2 *>(sXo)[n] = make_int2(0, 0);
+        else sXo[n] = 0;
     }
     if (half == 0) {   // warps 0 and 1: the edges that start their row, and whether a row
                        // without edges precedes any of them, one word each
@@ -481,8 +482,8 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
         const float b1f = A.b1[f], b2f = A.b2[f];
         const float *xbase = x_base(A, f), *hbase = A.Hbar + f;
-        const int *sXo = reinterpret_cast<const int *>(G.R + S::XO);
-        const int *sHo = reinterpret_cast<const int *>(G.R + S::HO);
+        const int2 *sOff = reinterpret_cast<const int2 *>(G.R + S::XO);
+        const uint32_t *sMask = reinterpret_cast<const uint32_t *>(G.R + S::MASK);
         const int *sDst = reinterpret_cast<const int *>(G.R + S::DST);
         const double *sDist = reinterpret_cast<const double *>(G.R + S::DIST);
         const float *sU = reinterpret_cast<const float *>(G.R + S::UVEC);
@@ -516,26 +517,36 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         };
         // xbar_i += hbar_j (.) (w + b2) and the tile of wbar = x_j (.) hbar_i + x_i (.) hbar_j over
         // one chunk of CH edges (zero for padding edges)
-        auto chunk = [&](int c, int ne, auto full) {
+        // A row changes exactly at the edges that start their row (the tile's row-start mask), so
+        // chunks without a start skip the row bookkeeping.
+        auto chunk = [&](int c, int ne, uint64_t starts, auto full) {
             constexpr bool FULL = decltype(full)::value;
             float w[CH], hb[CH], xj[CH];
             tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, w);
 #pragma unroll
             for (int q = 0; q < CH; ++q) {
-                const int n = CH * c + q;
-                hb[q] = __ldg(hbase + sHo[n]);
-                xj[q] = __ldg(xbase + sXo[n]);
+                const int2 o = sOff[CH * c + q];
+                xj[q] = __ldg(xbase + o.x);
+                hb[q] = __ldg(hbase + o.y);
             }
+            const uint32_t m = (uint32_t)(starts >> (CH * c)) & (CH >= 32 ? 0xffffffffu : (1u << (CH & 31)) - 1u);
+            if (FULL && m == 0) {
 #pragma unroll
-            for (int q = 0; q < CH; ++q) {
-                const int n = CH * c + q;
-                if (FULL || n < ne) {
-                    const int i = sDst[n];
-                    if (i != cur) next_row(i);
+                for (int q = 0; q < CH; ++q) {
                     xbacc = fmaf(hb[q], w[q] + b2f, xbacc);
                     xj[q] = xj[q] * hi_c + xi_c * hb[q];
-                } else {
-                    xj[q] = 0.0f;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < CH; ++q) {
+                    const int n = CH * c + q;
+                    if (FULL || n < ne) {
+                        if ((m >> q) & 1u) next_row(sDst[n]);
+                        xbacc = fmaf(hb[q], w[q] + b2f, xbacc);
+                        xj[q] = xj[q] * hi_c + xi_c * hb[q];
+                    } else {
+                        xj[q] = 0.0f;
+                    }
                 }
             }
             store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, xj);
@@ -554,10 +565,11 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
             if (more) npos = load_pos(A, nidx);
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
                 break;
+            const uint64_t starts = (uint64_t)sMask[0] | ((uint64_t)sMask[1] << 32);
 #pragma unroll 1
             for (int c = 0; c < TE / CH; ++c) {
-                if (CH * c + CH <= ne) chunk(c, ne, std::true_type{});
-                else chunk(c, ne, std::false_type{});
+                if (CH * c + CH <= ne) chunk(c, ne, starts, std::true_type{});
+                else chunk(c, ne, starts, std::false_type{});
             }
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, true>(sm, G.R, G.tm + COL_W); })))
                 break;
