@@ -214,11 +214,17 @@ __global__ void __launch_bounds__(1024) k_scan(const int32_t *__restrict__ in, i
     if (t == 0) out[0] = 0;
     long long carry = 0;
     bool over = false;
+    int nv[4];   // the next tile's entries, loaded while the current one is scanned
+#pragma unroll
+    for (int k = 0; k < 4; ++k) nv[k] = 4 * t + k < n ? in[4 * t + k] : 0;
     for (int64_t tile = 0; tile < n; tile += 4096) {
         const int64_t q0 = tile + 4 * t;
         int v[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) v[k] = q0 + k < n ? in[q0 + k] : 0;
+        for (int k = 0; k < 4; ++k) {
+            v[k] = nv[k];
+            nv[k] = q0 + 4096 + k < n ? in[q0 + 4096 + k] : 0;
+        }
         const long long s = (long long)v[0] + v[1] + v[2] + v[3];
         long long x = s;   // inclusive scan of the thread sums within the warp
 #pragma unroll

@@ -173,6 +173,12 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
+            float xr[32];   // the residual's x^t, loaded while the second GEMM runs
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const int64_t a = a0 + 32 * c + q;
+                xr[q] = a < A.N ? __ldg(x_row(A, A.t, a) + f) : 0.0f;
+            }
             if (!gemm_step<SPLIT, false>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar)) break;
             {
                 float v[32];
@@ -180,7 +186,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const int64_t a = a0 + 32 * c + q;
-                    if (a < A.N) A.X[((int64_t)A.t * A.N + a) * FF + f] = __ldg(x_row(A, A.t, a) + f) + v[q] + c2f;
+                    if (a < A.N) A.X[((int64_t)A.t * A.N + a) * FF + f] = xr[q] + v[q] + c2f;
                 }
             }
             tc_fence_before();
