@@ -904,19 +904,35 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                 auto chunk = [&](int c, auto full) {
                     constexpr bool FAST = decltype(full)::value;
                     float v[CH], xs[CH];
-                    int dst[CH];
                     tmem_ld<CH>(tmem + lanes + 64 * s + CH * c, v);
 #pragma unroll
-                    for (int q = 0; q < CH; ++q) {
-                        xs[q] = sXs[(CH * c + q) * FF];
-                        dst[q] = sDst[CH * c + q];
-                    }
+                    for (int q = 0; q < CH; ++q) xs[q] = sXs[(CH * c + q) * FF];
                     const uint32_t m = (uint32_t)(starts >> (CH * c)) & (CH >= 32 ? 0xffffffffu : (1u << (CH & 31)) - 1u);
                     if (FAST && m == 0) {   // the chunk continues the current row
 #pragma unroll
                         for (int q = 0; q < CH; ++q) hacc = fmaf(xs[q], v[q] + b2f, hacc);
                         return;
                     }
+                    if (FAST && (m & (m - 1u)) == 0) {
+                        // one row starts at edge p of the chunk: edges before it finish row cur,
+                        // edges from it open the next row (two running sums, one store)
+                        const int p = __ffs(m) - 1;
+                        float a0 = hacc, b0 = 0.0f;
+#pragma unroll
+                        for (int q = 0; q < CH; ++q) {
+                            const bool before = q < p;
+                            const float t0 = fmaf(xs[q], v[q] + b2f, before ? a0 : b0);
+                            a0 = before ? t0 : a0;
+                            b0 = before ? b0 : t0;
+                        }
+                        store_if(A.H + (int64_t)cur * FF + f, a0, true);
+                        cur = sDst[CH * c + p];
+                        hacc = b0;
+                        return;
+                    }
+                    int dst[CH];
+#pragma unroll
+                    for (int q = 0; q < CH; ++q) dst[q] = sDst[CH * c + q];
 #pragma unroll
                     for (int q = 0; q < CH; ++q) {
                         const int n = CH * c + q;
