@@ -556,11 +556,10 @@ sn_status md_run(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *vel_d
         cudaError_t e;
         if (lv)
             e = sn::launch_langevin_baoa(pos_dev, vel_dev, forces_dev, N, c, dt_fs, lv->a, lv->b, lv->seed,
-                                         lv->step0 + s, ctx->d_err, ctx->stream, &ctx->tracer);
+                                         lv->step0 + s, w.pos4, ctx->d_err, ctx->stream, &ctx->tracer);
         else
-            e = sn::launch_kick_drift(pos_dev, vel_dev, forces_dev, 3 * N, c, dt_fs, ctx->d_err, ctx->stream,
+            e = sn::launch_kick_drift(pos_dev, vel_dev, forces_dev, N, c, dt_fs, w.pos4, ctx->d_err, ctx->stream,
                                       &ctx->tracer);
-        if (e == cudaSuccess) e = sn::launch_prep_positions(pos_dev, w.pos4, N, ctx->d_err, ctx->stream, &ctx->tracer);
         if (e == cudaSuccess)
             e = sn::launch_neighbors(*sys, ctx->cfg.r_cut, w.pos4, w, rp, cl, ctx->md_cap, ctx->d_err, nullptr,
                                      ctx->stream, &ctx->tracer);

@@ -566,12 +566,27 @@ __global__ void k_partition(const int32_t *__restrict__ row_ptr, int64_t N, int 
     part[c] = (int32_t)lo;
 }
 
-// dst[e] = i for every edge e of row i (the tensor-core kernels read an edge's row directly),
-// one warp per row; an edge index outside the buffer latches the capacity condition instead.
-__global__ void k_row_index(const int32_t *__restrict__ row_ptr, int64_t N, int32_t *__restrict__ dst, int64_t cap,
-                            int *__restrict__ d_err)
+// Row partition (as k_partition) in the first part_blocks blocks; in the others, one warp per
+// row writes dst[e] = i for every edge e of row i (the tensor-core kernels read an edge's row
+// directly); an edge index outside the buffer latches the capacity condition instead.
+__global__ void k_partition_rows(const int32_t *__restrict__ row_ptr, int64_t N, int G, int32_t *__restrict__ part,
+                                 unsigned part_blocks, int32_t *__restrict__ dst, int64_t cap, int *__restrict__ d_err)
 {
-    const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
+    if (blockIdx.x < part_blocks) {
+        const int c = blockIdx.x * blockDim.x + threadIdx.x;
+        if (c > G) return;
+        const int64_t total = (int64_t)row_ptr[N] + N;
+        const int64_t target = (total * c + G - 1) / G;
+        int64_t lo = 0, hi = N;
+        while (lo < hi) {
+            const int64_t mid = (lo + hi) >> 1;
+            if ((int64_t)row_ptr[mid] + mid >= target) hi = mid;
+            else lo = mid + 1;
+        }
+        part[c] = (int32_t)lo;
+        return;
+    }
+    const int64_t i = ((blockIdx.x - part_blocks) * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (i >= N) return;
     const int32_t e0 = row_ptr[i], e1 = row_ptr[i + 1];
@@ -636,9 +651,14 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
 
     trace_begin(tr, KK_PARTITION, s);
     const int parts = m.precision == SN_PREC_FP32 ? w.G : w.G * tc_groups_per_cta(m.precision == SN_PREC_TC32);
-    k_partition<<<(parts + 1 + 127) / 128, 128, 0, s>>>(row_ptr, N, parts, w.part);
-    if (m.precision != SN_PREC_FP32 && N > 0)
-        k_row_index<<<(unsigned)((32 * N + 255) / 256), 256, 0, s>>>(row_ptr, N, w.dst, w.dst_cap, d_err);
+    if (m.precision != SN_PREC_FP32 && N > 0) {
+        // one launch: the first blocks partition the rows, the rest index the edges' rows
+        const unsigned pb = (unsigned)((parts + 1 + 255) / 256);
+        k_partition_rows<<<pb + (unsigned)((32 * N + 255) / 256), 256, 0, s>>>(row_ptr, N, parts, w.part, pb, w.dst,
+                                                                                w.dst_cap, d_err);
+    } else {
+        k_partition<<<(parts + 1 + 127) / 128, 128, 0, s>>>(row_ptr, N, parts, w.part);
+    }
     trace_end(tr, s);
 
     EdgeArgs ea{};

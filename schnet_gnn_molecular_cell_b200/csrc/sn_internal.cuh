@@ -190,13 +190,15 @@ struct NodeTcArgs {
 cudaError_t launch_node_tc(const NodeTcArgs &a, bool split, int which, int n_sm, cudaStream_t s);
 
 // ---------------------------------------------------------------- integrator
-cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t n3, float c,
-                              float dt, int *d_err, cudaStream_t s, Tracer *tr);
+cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t N, float c,
+                              float dt, float4 *pos4, int *d_err, cudaStream_t s, Tracer *tr);
 cudaError_t launch_kick(float *vel, const float *forces, int64_t n3, float c, int *d_err,
                         cudaStream_t s, Tracer *tr);
-// BAOAB first half (B, A, O, A) with Philox4x32-10 / Box-Muller noise keyed by (seed, step, atom)
+// BAOAB first half (B, A, O, A) with Philox4x32-10 / Box-Muller noise keyed by (seed, step, atom);
+// both drift kernels also refresh the float4 position copy (replacing launch_prep_positions)
 cudaError_t launch_langevin_baoa(float *pos, float *vel, const float *forces, int64_t N, float c, float dt, float a,
-                                 float b, uint64_t seed, int64_t step, int *d_err, cudaStream_t s, Tracer *tr);
+                                 float b, uint64_t seed, int64_t step, float4 *pos4, int *d_err, cudaStream_t s,
+                                 Tracer *tr);
 cudaError_t launch_replica_sums(const float *eps, const float *vel, int n_per, int n_rep,
                                 float half_m_over_kappa, float *energy, float *kinetic,
                                 int *d_err, cudaStream_t s, Tracer *tr);

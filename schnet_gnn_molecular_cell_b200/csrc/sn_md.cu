@@ -14,16 +14,35 @@ __device__ __forceinline__ bool skip_all(const int *d_err)
     return (*((volatile const int *)d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
 }
 
-// v += c F ; r += dt v   (c = dt/2 * kappa / m), per component
+// The drifted position also goes to the float4 copy the neighbour and edge kernels read
+// (a non-finite coordinate latches the condition and stores zeros there).
+__device__ __forceinline__ void store_pos4(float4 *pos4, int64_t i, const float (&x)[3], int *d_err)
+{
+    if (!isfinite(x[0]) || !isfinite(x[1]) || !isfinite(x[2])) {
+        atomicOr(d_err, ERRBIT_NONFINITE);
+        pos4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    } else {
+        pos4[i] = make_float4(x[0], x[1], x[2], 0.0f);
+    }
+}
+
+// v += c F ; r += dt v   (c = dt/2 * kappa / m), per atom
 __global__ void k_kick_drift(float *__restrict__ pos, float *__restrict__ vel, const float *__restrict__ forces,
-                             int64_t n3, float c, float dt, const int *__restrict__ d_err)
+                             int64_t N, float c, float dt, float4 *__restrict__ pos4, int *__restrict__ d_err)
 {
     if (skip_all(d_err)) return;
-    int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (q >= n3) return;
-    const float v = vel[q] + c * forces[q];
-    vel[q] = v;
-    pos[q] = pos[q] + dt * v;
+    const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+    if (i >= N) return;
+    float x[3];
+#pragma unroll
+    for (int d = 0; d < 3; ++d) {
+        const int64_t q = 3 * i + d;
+        const float v = vel[q] + c * forces[q];
+        vel[q] = v;
+        x[d] = pos[q] + dt * v;
+        pos[q] = x[d];
+    }
+    store_pos4(pos4, i, x, d_err);
 }
 
 __global__ void k_kick(float *__restrict__ vel, const float *__restrict__ forces, int64_t n3, float c,
@@ -109,12 +128,12 @@ __device__ __forceinline__ void langevin_noise(uint64_t seed, int64_t step, int6
 // BAOAB first half per atom: v += c F; r += dt/2 v; v = a v + b xi; r += dt/2 v
 __global__ void k_langevin_baoa(float *__restrict__ pos, float *__restrict__ vel, const float *__restrict__ forces,
                                 int64_t N, float c, float dt, float a, float b, uint64_t seed, int64_t step,
-                                const int *__restrict__ d_err)
+                                float4 *__restrict__ pos4, int *__restrict__ d_err)
 {
     if (skip_all(d_err)) return;
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= N) return;
-    float xi[3];
+    float xi[3], xn[3];
     langevin_noise(seed, step, i, xi);
 #pragma unroll
     for (int d = 0; d < 3; ++d) {
@@ -122,9 +141,11 @@ __global__ void k_langevin_baoa(float *__restrict__ pos, float *__restrict__ vel
         float v = vel[q] + c * forces[q];
         float x = pos[q] + 0.5f * dt * v;
         v = a * v + b * xi[d];
-        pos[q] = x + 0.5f * dt * v;
+        xn[d] = x + 0.5f * dt * v;
+        pos[q] = xn[d];
         vel[q] = v;
     }
+    store_pos4(pos4, i, xn, d_err);
 }
 
 inline unsigned blocks_for(int64_t n, int bt) { return (unsigned)((n + bt - 1) / bt); }
@@ -132,21 +153,22 @@ inline unsigned blocks_for(int64_t n, int bt) { return (unsigned)((n + bt - 1) /
 }  // namespace
 
 cudaError_t launch_langevin_baoa(float *pos, float *vel, const float *forces, int64_t N, float c, float dt, float a,
-                                 float b, uint64_t seed, int64_t step, int *d_err, cudaStream_t s, Tracer *tr)
+                                 float b, uint64_t seed, int64_t step, float4 *pos4, int *d_err, cudaStream_t s,
+                                 Tracer *tr)
 {
     if (N == 0) return cudaSuccess;
     trace_begin(tr, KK_KICK_DRIFT, s);
-    k_langevin_baoa<<<blocks_for(N, 128), 128, 0, s>>>(pos, vel, forces, N, c, dt, a, b, seed, step, d_err);
+    k_langevin_baoa<<<blocks_for(N, 128), 128, 0, s>>>(pos, vel, forces, N, c, dt, a, b, seed, step, pos4, d_err);
     trace_end(tr, s);
     return cudaGetLastError();
 }
 
-cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t n3, float c, float dt,
-                              int *d_err, cudaStream_t s, Tracer *tr)
+cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t N, float c, float dt,
+                              float4 *pos4, int *d_err, cudaStream_t s, Tracer *tr)
 {
-    if (n3 == 0) return cudaSuccess;
+    if (N == 0) return cudaSuccess;
     trace_begin(tr, KK_KICK_DRIFT, s);
-    k_kick_drift<<<blocks_for(n3, 256), 256, 0, s>>>(pos, vel, forces, n3, c, dt, d_err);
+    k_kick_drift<<<blocks_for(N, 256), 256, 0, s>>>(pos, vel, forces, N, c, dt, pos4, d_err);
     trace_end(tr, s);
     return cudaGetLastError();
 }
