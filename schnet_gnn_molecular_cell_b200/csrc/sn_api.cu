@@ -203,6 +203,7 @@ sn::EfWork ef_work(sn_ctx *ctx)
     w.part = (int32_t *)ctx->part.p;
     w.dst = (int32_t *)ctx->dst.p;
     w.dst_cap = (int64_t)(ctx->dst.bytes / sizeof(int32_t));
+    w.col_cap = 0;
     w.G = edge_grid(ctx);
     return w;
 }
@@ -239,9 +240,10 @@ sn_status drain(sn_ctx *ctx)
 
 // energy + forces on positions already staged in ctx->pos4
 sn_status enqueue_ef(sn_ctx *ctx, const sn_system *s, const int32_t *types, const int32_t *row_ptr,
-                     const int32_t *col, float *energy, float *forces)
+                     const int32_t *col, int64_t n_col, float *energy, float *forces)
 {
     sn::EfWork w = ef_work(ctx);
+    w.col_cap = n_col;
     const sn::Geometry g = geometry(s);
     cudaError_t e = sn::launch_energy_forces(ctx->model, *s, g, types, row_ptr, col, w, energy, forces,
                                              ctx->d_err, ctx->stream, &ctx->tracer);
@@ -505,7 +507,7 @@ sn_status sn_energy_forces(sn_ctx *ctx, const sn_system *sys, const float *pos_d
     if ((st = grow(ctx, ctx->dst, sizeof(int32_t) * (size_t)n_edges))) return st;
     cudaError_t e = sn::launch_prep_positions(pos_dev, (float4 *)ctx->pos4.p, N, ctx->d_err, ctx->stream, &ctx->tracer);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "prep positions");
-    return enqueue_ef(ctx, sys, types_dev, row_ptr_dev, col_dev, energy_dev, forces_dev);
+    return enqueue_ef(ctx, sys, types_dev, row_ptr_dev, col_dev, n_edges, energy_dev, forces_dev);
 }
 
 }  // extern "C"
@@ -565,6 +567,7 @@ sn_status md_run(sn_ctx *ctx, const sn_system *sys, float *pos_dev, float *vel_d
                                      ctx->stream, &ctx->tracer);
         if (e != cudaSuccess) return cuda_fail(ctx, e, "md step: drift / neighbours");
         sn::EfWork ew = ef_work(ctx);
+        ew.col_cap = ctx->md_cap;
         e = sn::launch_energy_forces(ctx->model, *sys, geometry(sys), types_dev, rp, cl, ew, nullptr, forces_dev,
                                      ctx->d_err, ctx->stream, &ctx->tracer);
         if (e == cudaSuccess) e = sn::launch_kick(vel_dev, forces_dev, 3 * N, c, ctx->d_err, ctx->stream, &ctx->tracer);

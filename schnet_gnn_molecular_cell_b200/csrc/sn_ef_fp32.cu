@@ -551,9 +551,13 @@ __global__ void __launch_bounds__(F) k_node_bwd(NodeArgs A)
     }
 }
 
-__global__ void k_partition(const int32_t *__restrict__ row_ptr, int64_t N, int G, int32_t *__restrict__ part)
+// Also checks that the list fits the caller's col buffer (cap entries): a row_ptr that points
+// past it latches the capacity condition, and every later kernel skips.
+__global__ void k_partition(const int32_t *__restrict__ row_ptr, int64_t N, int G, int32_t *__restrict__ part,
+                            int64_t cap, int *__restrict__ d_err)
 {
     const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c == 0 && (row_ptr[0] < 0 || (int64_t)row_ptr[N] > cap)) atomicOr(d_err, ERRBIT_CAPACITY);
     if (c > G) return;
     const int64_t total = (int64_t)row_ptr[N] + N;
     const int64_t target = (total * c + G - 1) / G;
@@ -654,10 +658,10 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
     if (m.precision != SN_PREC_FP32 && N > 0) {
         // one launch: the first blocks partition the rows, the rest index the edges' rows
         const unsigned pb = (unsigned)((parts + 1 + 255) / 256);
-        k_partition_rows<<<pb + (unsigned)((32 * N + 255) / 256), 256, 0, s>>>(row_ptr, N, parts, w.part, pb, w.dst,
-                                                                                w.dst_cap, d_err);
+        k_partition_rows<<<pb + (unsigned)((32 * N + 255) / 256), 256, 0, s>>>(
+            row_ptr, N, parts, w.part, pb, w.dst, w.col_cap < w.dst_cap ? w.col_cap : w.dst_cap, d_err);
     } else {
-        k_partition<<<(parts + 1 + 127) / 128, 128, 0, s>>>(row_ptr, N, parts, w.part);
+        k_partition<<<(parts + 1 + 127) / 128, 128, 0, s>>>(row_ptr, N, parts, w.part, w.col_cap, d_err);
     }
     trace_end(tr, s);
 

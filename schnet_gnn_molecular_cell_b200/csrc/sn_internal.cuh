@@ -127,6 +127,7 @@ struct EfWork {
     int32_t *part;       // [4 G + 1]   rows owned by each CTA (fp32) / warpgroup (tensor cores)
     int32_t *dst;        // [dst_cap]   destination row of every edge (tensor-core kernels)
     int64_t dst_cap;
+    int64_t col_cap;     // entries of this call's col buffer (the list must fit in it)
     int G;
 };
 

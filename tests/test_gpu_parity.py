@@ -176,3 +176,22 @@ def test_invalid_box_and_sizes(dev):
     with pytest.raises(SNError) as ei:
         ctx.neighbors(s, torch.zeros((10, 3), dtype=torch.float32, device=dev))
     assert ei.value.status == Status.INVALID_ARG
+
+
+@pytest.mark.parametrize("precision", [0, 1, 2])
+def test_list_longer_than_col_is_reported(oracle, dev, precision):
+    # a row_ptr whose last entry points past the col buffer handed in: capacity status, no
+    # kernel reads past the buffer, and the context stays usable
+    from schnet_gnn_molecular_cell_b200 import Context, SNError, Status
+    w = synth.make_workload(4)
+    ctx = Context(w.model, w.weights, precision=precision)
+    rp, cl = oracle.neighbors(w.system, w.model.r_cut, w.pos, "cells")
+    pos, types = to_dev(w.pos, dev), to_dev(w.types, dev)
+    short = to_dev(cl[: len(cl) // 2], dev)
+    ctx.energy_forces(w.system, pos, types, to_dev(rp, dev), short)
+    with pytest.raises(SNError) as ei:
+        ctx.sync()
+    assert ei.value.status == Status.CAPACITY
+    E, F = ctx.energy_forces(w.system, pos, types, to_dev(rp, dev), to_dev(cl, dev))
+    ctx.sync()
+    assert np.isfinite(F.cpu().numpy()).all()
