@@ -144,7 +144,9 @@ sn_status sn_build_neighbors(sn_ctx *ctx, const sn_system *sys, const float *pos
  *   row_ptr_dev int32 [N+1], col_dev int32 [n_edges] (n_edges = row_ptr[N]);
  *   energy_dev float32 [n_replicas] (out), forces_dev float32 [N][3] (out).
  * The list must be symmetric (j -> i present iff i -> j present), as sn_build_neighbors
- * produces; the force kernel relies on it.  Asynchronous.
+ * produces; the force kernel relies on it.  Asynchronous: a row_ptr whose last entry
+ * exceeds n_edges (or whose first is negative) is detected on the device before col is
+ * read, and the next sn_sync returns SN_ERR_CAPACITY (outputs unspecified).
  */
 sn_status sn_energy_forces(sn_ctx *ctx, const sn_system *sys, const float *pos_dev,
                            const int32_t *types_dev, const int32_t *row_ptr_dev,
