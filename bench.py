@@ -46,7 +46,7 @@ WORKLOAD = "64 x 269-bead SAW chains, r_cut 12 A, SchNet F128 K50 T3: one veloci
            "(neighbour rebuild + energy/forces + integration)"
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
@@ -61,7 +61,19 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="replica-scaling sweep instead of the benchmark line: one JSON line per "
                          "(replicas, chain kind) with evals/s, steps x replicas/s and workspace bytes")
-    return ap.parse_args()
+    return ap.parse_args(argv)
+
+
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of a per-rank number over all ranks of the process group (the number itself
+    with one rank): per-step times are reported as the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def dist_env():
@@ -304,11 +316,9 @@ def run_ours(args):
     ctx.trace(False)
     ctx.sync()
     E_tr /= n_tr
+    t_ms = max_over_ranks(t_ms, dev)
     if world > 1:
-        t = torch.tensor([t_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         torch.distributed.barrier()
-        t_ms = float(t.item())
     E_mean = 0.5 * (E_start + E_end)
     value = world * args.steps / (t_ms / 1e3)
 
@@ -351,10 +361,7 @@ def run_ours(args):
             t1 = time.perf_counter()
             if k >= 2:
                 tot += t1 - t0
-        if world > 1:
-            t = torch.tensor([tot], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            tot = float(t.item())
+        tot = max_over_ranks(tot, dev)
         e2e = {"value": world * n_e2e / tot, "unit": "evals/s",
                "h2d_bytes_per_step": 3 * (3 * N * 4) + N * 4,
                "d2h_bytes_per_step": 3 * (3 * N * 4) + 2 * R * 4,
