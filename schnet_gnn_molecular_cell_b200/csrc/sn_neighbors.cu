@@ -258,6 +258,84 @@ __global__ void __launch_bounds__(1024) k_scan(const int32_t *__restrict__ in, i
     if (over) atomicOr(d_err, ERRBIT_CAPACITY);
 }
 
+// The same exclusive scan over many CTAs, in two launches: k_scan_tiles scans each 4096-entry
+// tile in its own CTA (tile-local sums into out, tile totals into tsum); k_scan_add adds the
+// totals of the earlier tiles.  Used where a scratch array of ceil(n / 4096) entries is free.
+__device__ __forceinline__ long long block_scan_1024(long long s, long long &total, long long *warp_sums)
+{
+    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+    long long x = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[wid] = x;
+    __syncthreads();
+    if (wid == 0) {
+        long long ws = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const long long y = __shfl_up_sync(0xffffffffu, ws, o);
+            if (lane >= o) ws += y;
+        }
+        warp_sums[lane] = ws;
+    }
+    __syncthreads();
+    total = warp_sums[31];
+    return x - s + (wid > 0 ? warp_sums[wid - 1] : 0);   // exclusive prefix of s
+}
+
+__global__ void __launch_bounds__(1024) k_scan_tiles(const int32_t *__restrict__ in, int32_t *__restrict__ out,
+                                                     int64_t n, int32_t *__restrict__ tsum)
+{
+    __shared__ long long warp_sums[32];
+    const int t = threadIdx.x;
+    const int64_t q0 = (int64_t)blockIdx.x * 4096 + 4 * t;
+    int v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = q0 + k < n ? in[q0 + k] : 0;
+    long long total;
+    long long run = block_scan_1024((long long)v[0] + v[1] + v[2] + v[3], total, warp_sums);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        if (q0 + k < n) {
+            run += v[k];
+            out[q0 + k + 1] = (int32_t)(run > 0x7fffffffLL ? 0x7fffffff : run);
+        }
+    if (t == 0) {
+        tsum[blockIdx.x] = (int32_t)(total > 0x7fffffffLL ? 0x7fffffff : total);
+        if (blockIdx.x == 0) out[0] = 0;
+    }
+}
+
+__global__ void __launch_bounds__(1024) k_scan_add(int32_t *__restrict__ out, int64_t n,
+                                                   const int32_t *__restrict__ tsum, int *__restrict__ d_err)
+{
+    __shared__ long long part[32];
+    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
+    long long off = 0;
+    for (int b = t; b < (int)blockIdx.x; b += 1024) off += tsum[b];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
+    if (lane == 0) part[wid] = off;
+    __syncthreads();
+    off = 0;
+#pragma unroll 1
+    for (int w = 0; w < 32; ++w) off += part[w];
+    if (off == 0) return;
+    const int64_t q0 = (int64_t)blockIdx.x * 4096 + 4 * t;
+    bool over = false;
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        if (q0 + k < n) {
+            const long long v = off + out[q0 + k + 1];
+            over |= v > 0x7fffffffLL;
+            out[q0 + k + 1] = (int32_t)(v > 0x7fffffffLL ? 0x7fffffff : v);
+        }
+    if (__any_sync(0xffffffffu, over) && lane == 0) atomicOr(d_err, ERRBIT_CAPACITY);
+}
+
 __global__ void k_copy_i32(const int32_t *__restrict__ a, int32_t *__restrict__ b, int64_t n)
 {
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
@@ -341,7 +419,13 @@ cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *po
         trace_end(tr, s);
     }
     trace_begin(tr, KK_SCAN, s);
-    k_scan<<<1, 1024, 0, s>>>(w.cnt, row_ptr, N, d_err);
+    if (!cells) {   // row offsets over many CTAs (cell_of is free scratch on this path)
+        const unsigned tiles = (unsigned)((N + 4095) / 4096);
+        k_scan_tiles<<<tiles, 1024, 0, s>>>(w.cnt, row_ptr, N, w.cell_of);
+        k_scan_add<<<tiles, 1024, 0, s>>>(row_ptr, N, w.cell_of, d_err);
+    } else {
+        k_scan<<<1, 1024, 0, s>>>(w.cnt, row_ptr, N, d_err);
+    }
     trace_end(tr, s);
     if ((e = cudaGetLastError())) return e;
     if (n_edges_host) {
