@@ -41,6 +41,7 @@ MASS, DT, TEMP = 12.0, 2.0, 300.0
 # name -> (ABI precision, dtype string, tensor MMAs per algorithmic product)
 PRECISIONS = {"tc32": (2, "f16x2-split (fp32-accurate), f32 accumulate", 3),
               "fp16": (1, "f16, f32 accumulate", 1),
+              "fp16_ch": (3, "f16 with per-output-channel weight scales, f32 accumulate", 1),
               "fp32": (0, "f32", 0)}
 WORKLOAD = "64 x 269-bead SAW chains, r_cut 12 A, SchNet F128 K50 T3: one velocity-Verlet step " \
            "(neighbour rebuild + energy/forces + integration)"
@@ -58,6 +59,8 @@ def parse(argv=None):
                     help="network arithmetic: fp16 = fp16 operands on tensor cores, fp32 accumulate "
                          "(W16A16, default), tc32 = fp32-accurate fp16 split on tensor cores, fp32 = CUDA cores")
     ap.add_argument("--no-variants", action="store_true", help="skip the short runs of the other precisions")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the cfg4 / evaluation-only rooflines and the cfg3 1000-step drift runs")
     ap.add_argument("--sweep", action="store_true",
                     help="replica-scaling sweep instead of the benchmark line: one JSON line per "
                          "(replicas, chain kind) with evals/s, steps x replicas/s and workspace bytes")
@@ -82,10 +85,37 @@ def dist_env():
 
 
 # ------------------------------------------------------------------------------ CPU oracle
-def oracle_md_rate(w, v0, n_rep_sample: int, budget_s: float, min_steps: int = 1):
+_NATIVE = None
+
+
+def native_oracle():
+    """The oracle built for this host (-O3 -march=native, same IEEE semantics), compiled here
+    at run time into oracle/_build; the build used by every timed CPU leg."""
+    global _NATIVE
+    if _NATIVE is None:
+        from oracle import oracle
+        d = ROOT / "oracle" / "_build"
+        d.mkdir(exist_ok=True)
+        _NATIVE = oracle.build_native(d)
+    return _NATIVE
+
+
+def oracle_md_rate(w, v0, n_rep_sample: int, budget_s: float, min_steps: int = 1, threads: int | None = None):
     """Time the CPU oracle's velocity-Verlet steps on the first n_rep_sample replicas of the
-    workload; returns (evals/s scaled to the full workload, steps run, seconds, threads)."""
+    workload (native build; `threads` OpenMP threads, default all); returns (evals/s scaled to
+    the full workload, steps run, seconds, threads)."""
     from oracle import oracle
+    with oracle.using(native_oracle()):
+        n0 = oracle.num_threads()
+        if threads is not None:
+            oracle.set_threads(threads)
+        try:
+            return _oracle_md_rate(oracle, w, v0, n_rep_sample, budget_s, min_steps)
+        finally:
+            oracle.set_threads(n0)
+
+
+def _oracle_md_rate(oracle, w, v0, n_rep_sample, budget_s, min_steps):
     n_per = w.system.n_per_replica
     s = synth.SystemCfg(n_per, n_rep_sample, w.system.box)
     n = n_per * n_rep_sample
@@ -119,6 +149,7 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": rate, "unit": "evals/s", "cores": threads, "kind": "oracle",
+                         "build": "gcc -O3 -march=native -fopenmp -ffp-contract=off",
                          "sample": f"{n_sample} of {s.n_replicas} replicas per step, {steps} steps in "
                                    f"{secs:.1f} s; rate scaled to the full batch"},
         "e2e": {"value": rate, "unit": "evals/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -199,6 +230,123 @@ def kernel_traffic(kernel: str, src: Path, precision: str = "fp32"):
                 and parts.get("precision", "fp32") == precision):
             return float(parts["bytes_per_launch"])
     return None
+
+
+# ------------------------------------------------------------------------------ whole-evaluation roofline
+def eval_roofline(m, N: int, E: float, t_s: float, pk: dict, build: bool = False) -> dict:
+    """One evaluation (or MD step, build=True) against the roof of the whole path: the slower of
+    the minimum fused HBM bytes at the measured copy bandwidth and the filter networks'
+    algorithmic FLOPs at the measured sustained dense tensor peak.
+      FLOPs: 4 (K F + F^2) per directed edge per block (forward K->F->F, backward F->F->K).
+      bytes: per block 8 passes over an [N][F] fp32 array (x read and written, h saved, hbar
+             written and read, xbar read and written, p saved) = 32 N F, plus the 4-byte source
+             and destination index of every edge; once per evaluation positions in, types,
+             forces out (28 N); an MD step adds the list build (positions in, 4-byte counts and
+             row offsets, the 4-byte col of every edge) and the integrator's 5 passes over
+             [N][3] fp32 arrays."""
+    F, K, T = m.F, m.K, m.T
+    flops = 4.0 * (K * F + F * F) * E * T
+    nbytes = 32.0 * N * F * T + 8.0 * E * T + 28.0 * N
+    if build:
+        nbytes += 12.0 * N + 8.0 * N + 4.0 * E + 60.0 * N
+    t_hbm = nbytes / (pk["hbm_gbs"] * 1e9)
+    t_tc = flops / (pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) * 1e12)
+    t_roof = max(t_hbm, t_tc)
+    return {"bound": "tensor" if t_tc >= t_hbm else "hbm", "frac": t_roof / t_s,
+            "per_s": 1.0 / t_s, "roof_per_s": 1.0 / t_roof, "edges_per_s": E / t_s, "roof_edges_per_s": E / t_roof,
+            "flops": flops, "bytes": nbytes, "t_roof_us": t_roof * 1e6, "t_us": t_s * 1e6,
+            "peaks": f"{pk['hbm_gbs']:.0f} GB/s, {pk.get('bf16_tflops_sustained', pk['bf16_tflops']):.0f} TFLOP/s"}
+
+
+def time_evals(cfg: int, precision_code: int, steps: int, dev, stream, flush):
+    """Energy + forces alone on one configuration (list built once, outside the timing): CUDA
+    events around each evaluation on the library's stream, L2 flushed before each.  Returns
+    (seconds per evaluation, N, E, model)."""
+    import torch
+    from schnet_gnn_molecular_cell_b200 import Context
+    w = synth.make_workload(cfg)
+    s, m = w.system, w.model
+    ctx = Context(m, w.weights, stream=stream, precision=precision_code)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    types = torch.from_numpy(w.types).to(dev)
+    rp, cl = ctx.neighbors(s, pos)
+    energy = torch.empty(s.n_replicas, device=dev)
+    forces = torch.empty((s.n_atoms, 3), device=dev)
+    for q in range(3):
+        flush.fill_(float(q))
+        ctx.energy_forces(s, pos, types, rp, cl, energy, forces)
+    ctx.sync()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for q in range(steps):
+        flush.fill_(float(q))
+        ev[q][0].record(stream)
+        ctx.energy_forces(s, pos, types, rp, cl, energy, forces)
+        ev[q][1].record(stream)
+    torch.cuda.synchronize()
+    ctx.sync()
+    t = sum(a.elapsed_time(b) for a, b in ev) / steps / 1e3
+    ctx.close()
+    return t, s.n_atoms, int(cl.numel()), m
+
+
+def nve_drift(w, v0, precision_code: int, n_steps: int, dev, stream):
+    """cfg3: n_steps of velocity Verlet (dt 2 fs, 12 amu, list rebuilt every step) from the
+    seeded start; total energy E_pot + E_kin per replica after every step.  Returns the drift
+    figures: max_t |E_tot(t) - E_tot(0)| / (n k_B T) per replica (median and max over
+    replicas) and the slope of a linear fit of the replica-mean E_tot / (n k_B T) against
+    time, per ns."""
+    import torch
+    from schnet_gnn_molecular_cell_b200 import Context
+    s, m = w.system, w.model
+    R, n = s.n_replicas, s.n_per_replica
+    ctx = Context(m, w.weights, stream=stream, precision=precision_code)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.from_numpy(v0.copy()).to(dev)
+    types = torch.from_numpy(w.types).to(dev)
+    rp, cl = ctx.neighbors(s, pos)
+    e0, forces = ctx.energy_forces(s, pos, types, rp, cl)
+    forces = forces.clone()
+    ctx.reserve(s, 2 * int(cl.numel()) + 4096)
+    hist = torch.empty((n_steps, 2, R), device=dev)   # potential and kinetic after each step
+    t0 = time.perf_counter()
+    for k in range(n_steps):
+        ctx.md_step(s, pos, vel, forces, types, MASS, DT, 1, hist[k, 0], hist[k, 1])
+    ctx.sync()
+    wall = time.perf_counter() - t0
+    h = hist.double().cpu().numpy()
+    k0 = 0.5 * MASS / synth.KAPPA * (v0.astype(np.float64).reshape(R, n, 3) ** 2).sum(axis=(1, 2))
+    etot = np.vstack([e0.double().cpu().numpy() + k0, h[:, 0] + h[:, 1]])
+    ctx.close()
+    return drift_figures(etot, n, n_steps, wall), etot
+
+
+def drift_figures(etot, n_per: int, n_steps: int, wall_s: float | None = None) -> dict:
+    kT = synth.KB * TEMP
+    rel = (etot - etot[:1]) / (n_per * kT)             # [steps + 1][R]
+    per_rep = np.abs(rel).max(axis=0)
+    t_ns = np.arange(etot.shape[0]) * DT * 1e-6
+    slope = float(np.polyfit(t_ns, rel.mean(axis=1), 1)[0])
+    out = {"steps": n_steps, "dt_fs": DT, "max_abs_drift_per_nkT": {"median": float(np.median(per_rep)),
+                                                                    "max": float(per_rep.max())},
+           "slope_per_ns_per_nkT": slope}
+    if wall_s is not None:
+        out["wall_s"] = wall_s
+    return out
+
+
+def oracle_drift(w, v0, n_rep: int, n_steps: int) -> dict:
+    """The oracle's (double-precision) velocity-Verlet drift on the first n_rep replicas."""
+    from oracle import oracle
+    n = w.system.n_per_replica
+    s = synth.SystemCfg(n, n_rep, w.system.box)
+    with oracle.using(native_oracle()):
+        _, _, _, epot, ekin, _ = oracle.md_vv(w.model, w.weights, s, w.pos[: n * n_rep], v0[: n * n_rep],
+                                              w.types[: n * n_rep], MASS, DT, n_steps)
+        rp, cl = oracle.neighbors(s, w.model.r_cut, w.pos[: n * n_rep])
+        e0, _, _ = oracle.energy_forces(w.model, w.weights, s, w.pos[: n * n_rep], w.types[: n * n_rep], rp, cl)
+    k0 = 0.5 * MASS / synth.KAPPA * (v0[: n * n_rep].astype(np.float64).reshape(n_rep, n, 3) ** 2).sum(axis=(1, 2))
+    etot = np.vstack([e0 + k0, epot + ekin])
+    return drift_figures(etot, n, n_steps)
 
 
 # ------------------------------------------------------------------------------ our arm
@@ -370,8 +518,35 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, steps, secs, threads = oracle_md_rate(w, v0, R, 10.0)
+        r1, steps1, secs1, _ = oracle_md_rate(w, v0, 4, 8.0, threads=1)
         cpu = {"value": rate, "unit": "evals/s", "cores": threads, "kind": "oracle",
-               "sample": f"{steps} full velocity-Verlet step(s) of all {R} replicas in {secs:.1f} s"}
+               "build": "gcc -O3 -march=native -fopenmp -ffp-contract=off",
+               "sample": f"{steps} full velocity-Verlet step(s) of all {R} replicas in {secs:.1f} s",
+               "single_thread": {"value": r1, "unit": "evals/s", "cores": 1,
+                                 "sample": f"{steps1} step(s) of 4 of {R} replicas in {secs1:.1f} s, "
+                                           f"rate scaled to the full batch"}}
+
+    extras = {}
+    if rank == 0 and world == 1 and not args.no_extras:
+        # the 4096-atom periodic box (cfg4) and the chains' evaluation alone, each mode; the
+        # whole-evaluation roofline of these and of the MD step timed above
+        extras["roofline_eval"] = {"cfg2_md_step": eval_roofline(m, N, E_mean, t_ms / args.steps / 1e3, pk, build=True)}
+        extras["roofline_eval"]["cfg2_md_step"]["steps_x_replicas_per_s"] = value * R
+        extras["roofline_eval"]["cfg2_md_step"]["roof_steps_x_replicas_per_s"] = \
+            extras["roofline_eval"]["cfg2_md_step"]["roof_per_s"] * R
+        for cfg in (2, 4):
+            for name in ("fp16", "tc32"):
+                t_e, n_e, e_e, m_e = time_evals(cfg, PRECISIONS[name][0], 50, dev, stream, flush)
+                extras["roofline_eval"][f"cfg{cfg}_eval_{name}"] = eval_roofline(m_e, n_e, e_e, t_e, pk)
+        # cfg3: 1000 NVE steps of the chains in each tensor mode, total-energy drift; the
+        # oracle's over the first 100 steps of 4 replicas beside the same window of the GPU run
+        drift = {}
+        for name in ("fp16", "tc32"):
+            fig, etot = nve_drift(w, v0, PRECISIONS[name][0], 1000, dev, stream)
+            fig["first_100_steps_replicas_0_3"] = drift_figures(etot[:101, :4], s.n_per_replica, 100)
+            drift[name] = fig
+        drift["oracle_first_100_steps_replicas_0_3"] = oracle_drift(w, v0, 4, 100)
+        extras["nve_drift_cfg3"] = drift
 
     variants = None
     if rank == 0 and world == 1 and not args.no_variants:
@@ -398,6 +573,7 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": round(sum(v[0] for v in trace.values()) * args.steps / n_tr),
             "precision_variants": variants,
+            **extras,
             "clocks": clocks,
             "kernels": {k: {"launches": v[0], "ms_per_launch": v[1] / v[0], "share": v[1] / sum(x[1] for x in trace.values())}
                         for k, v in sorted(trace.items(), key=lambda kv: -kv[1][1])},

@@ -53,17 +53,27 @@ typedef enum {
     SN_ERR_TIMEOUT = 8        /* a kernel gave up waiting for its own tensor-core work      */
 } sn_status;
 
-/* Arithmetic of the filter network (update and readout networks are fp32 in all modes).
+/* Arithmetic of the MLPs: filter, update and readout networks alike (every GEMM of a mode
+ * uses the same operand precision; positions, distances, the Gaussian basis, energies,
+ * forces and all reductions are fp32, or double where stated, in every mode).
  *  SN_PREC_FP32: fp32 on CUDA cores.
- *  SN_PREC_FP16: fp16 operands on the tensor cores (tcgen05), fp32 accumulation in TMEM --
- *                the W16A16 precision of FlashSchNet §4.4 (per-tensor, no calibration).
+ *  SN_PREC_FP16: fp16 operands (weights and activations) on the tensor cores (tcgen05),
+ *                fp32 accumulation in TMEM -- the W16A16 precision of FlashSchNet §4.4,
+ *                weights cast to fp16 with round-to-nearest (one scale per tensor = 1).
  *  SN_PREC_TC32: fp32-accurate on the tensor cores: every operand split into two fp16
  *                terms, products accumulated as hi*hi + hi*lo + lo*hi (3 MMAs).
+ *  SN_PREC_FP16_CH: SN_PREC_FP16 with one scale per output channel (FlashSchNet §4.4
+ *                "channel-wise quantization"): every weight matrix W (W1, W2, U1, U2, R1) is
+ *                stored as fp16(W[o][:] / s_o), s_o = max_i |W[o][i]| (1 for an all-zero
+ *                row), and s_o multiplies the fp32 accumulator of output channel o; the
+ *                transposed products of the backward pass take s_o on their operand instead.
+ *                The scales are computed from the weights at sn_create (no calibration data).
  * The tensor-core modes need F = 128. */
 enum {
     SN_PREC_FP32 = 0,
     SN_PREC_FP16 = 1,
-    SN_PREC_TC32 = 2
+    SN_PREC_TC32 = 2,
+    SN_PREC_FP16_CH = 3
 };
 
 /* Model hyper-parameters.  Supported: F in {64, 128}, 2 <= K <= 64, T >= 1, n_types >= 1. */
@@ -218,10 +228,12 @@ sn_status sn_sync(sn_ctx *ctx);
  * the library keeps until the process exits.  Limits: at most SN_NOALLOC_MAX_ATOMS atoms
  * in total and, for periodic boxes built with the cell list, at most SN_NOALLOC_MAX_CELLS
  * cells (n_replicas x cells per box); larger systems get SN_ERR_UNSUPPORTED and nothing
- * is launched.  The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.  All calls share
- * the one array: calls that overlap on the GPU (different streams or host threads at the
- * same time) race and must be serialised by the caller.
+ * is launched.  Every call looks up the array's device address on the current device (a
+ * host-side lookup, repeated each call so that an address from before a cudaDeviceReset is
+ * never reused); the first call on a device also loads the library's device code there,
+ * so make that first call before any stream capture.  All calls share the one array:
+ * calls that overlap on the GPU (different streams or host threads at the same time) race
+ * and must be serialised by the caller.
  */
 #define SN_NOALLOC_MAX_ATOMS 65536
 #define SN_NOALLOC_MAX_CELLS 65536

@@ -20,7 +20,24 @@ SRC = HERE / "sn_oracle.c"
 LIB = HERE / "libsn_oracle.so"
 CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC"]
 
+# The build timed as the benchmark's CPU baseline: the same source and the same IEEE
+# semantics (no contraction, no fast-math), optimised for the host it runs on.  Compiled on
+# that host at run time, never shipped, so -march=native cannot meet a CPU it was not built for.
+NATIVE_CFLAGS = ["-O3", "-march=native", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-shared", "-fPIC"]
+
 _lib = None
+
+
+def build_native(out_dir: Path) -> Path:
+    """Compile the oracle with NATIVE_CFLAGS into out_dir (for the CPU-baseline timing)."""
+    out = Path(out_dir) / "libsn_oracle_native.so"
+    subprocess.check_call(["gcc", *NATIVE_CFLAGS, "-o", str(out), str(SRC), "-lm"])
+    return out
+
+
+def set_threads(n: int) -> None:
+    """OpenMP thread count of the oracle's later parallel regions (the process's libgomp)."""
+    C.CDLL("libgomp.so.1").omp_set_num_threads(C.c_int(int(n)))
 
 
 def build(force: bool = False) -> Path:

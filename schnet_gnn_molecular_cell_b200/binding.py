@@ -14,7 +14,11 @@ import numpy as np
 
 LIB_PATH = Path(__file__).resolve().parent / "libsnflash.so"
 
-PREC_FP32 = 0
+# network arithmetic (sn_config.precision; see include/sn.h)
+PREC_FP32 = 0      # CUDA-core fp32
+PREC_FP16 = 1      # fp16 operands on the tensor cores, fp32 accumulation (weights cast as they are)
+PREC_TC32 = 2      # fp32-accurate tensor-core split (hi + lo fp16 terms)
+PREC_FP16_CH = 3   # fp16 operands with one scale per output channel of every weight matrix
 
 
 class Status(enum.IntEnum):
@@ -26,6 +30,7 @@ class Status(enum.IntEnum):
     CUDA = 5
     UNSUPPORTED = 6
     NOMEM = 7
+    TIMEOUT = 8
 
 
 class SNError(RuntimeError):
@@ -112,10 +117,27 @@ def _ptr(t) -> int | None:
     return t.data_ptr() if t.numel() else None
 
 
-def _dev_check(t, dtype, name):
+def _dev_check(t, dtype, name, min_numel: int = 0):
+    """A contiguous tensor of `dtype` on the current CUDA device (the device whose stream and
+    buffers the library uses) with at least min_numel elements; else TypeError / SNError
+    (INVALID_ARG) before anything is handed to the library."""
     import torch
     if not (isinstance(t, torch.Tensor) and t.is_cuda and t.dtype == dtype and t.is_contiguous()):
         raise TypeError(f"{name} must be a contiguous CUDA tensor of {dtype}")
+    if t.device.index != torch.cuda.current_device():
+        raise SNError(Status.INVALID_ARG, f"{name} is on {t.device}, the current device is "
+                                          f"cuda:{torch.cuda.current_device()}")
+    if t.numel() < min_numel:
+        raise SNError(Status.INVALID_ARG, f"{name} has {t.numel()} elements, needs at least {min_numel}")
+
+
+def _check_md_arrays(system, pos, vel, forces, types, energy, kinetic):
+    import torch
+    N, R = system.n_per_replica * system.n_replicas, system.n_replicas
+    for t, dtp, n, k in ((pos, torch.float32, "pos", 3 * N), (vel, torch.float32, "vel", 3 * N),
+                         (forces, torch.float32, "forces", 3 * N), (types, torch.int32, "types", N),
+                         (energy, torch.float32, "energy", R), (kinetic, torch.float32, "kinetic", R)):
+        _dev_check(t, dtp, n, k)
 
 
 class Context:
@@ -162,8 +184,9 @@ class Context:
         """Fill row_ptr [N+1] / col [cap] (int32 CUDA tensors); returns E.  Raises SNError
         with status CAPACITY (and .needed = E) if col is too small."""
         import torch
-        _dev_check(pos, torch.float32, "pos")
-        _dev_check(row_ptr, torch.int32, "row_ptr")
+        N = system.n_per_replica * system.n_replicas
+        _dev_check(pos, torch.float32, "pos", 3 * N)
+        _dev_check(row_ptr, torch.int32, "row_ptr", N + 1)
         _dev_check(col, torch.int32, "col")
         ne = C.c_int64(0)
         st = self._L.sn_build_neighbors(self._h, C.byref(system_struct(system)), _ptr(pos), _ptr(row_ptr),
@@ -198,10 +221,13 @@ class Context:
             energy = torch.empty(system.n_replicas, dtype=torch.float32, device=pos.device)
         if forces is None:
             forces = torch.empty((N, 3), dtype=torch.float32, device=pos.device)
-        for t, dt, n in ((pos, torch.float32, "pos"), (types, torch.int32, "types"),
-                         (row_ptr, torch.int32, "row_ptr"), (energy, torch.float32, "energy"),
-                         (forces, torch.float32, "forces")):
-            _dev_check(t, dt, n)
+        R = system.n_replicas
+        for t, dt, n, k in ((pos, torch.float32, "pos", 3 * N), (types, torch.int32, "types", N),
+                            (row_ptr, torch.int32, "row_ptr", N + 1), (energy, torch.float32, "energy", R),
+                            (forces, torch.float32, "forces", 3 * N)):
+            _dev_check(t, dt, n, k)
+        if col.numel():
+            _dev_check(col, torch.int32, "col")
         self._check(self._L.sn_energy_forces(self._h, C.byref(system_struct(system)), _ptr(pos), _ptr(types),
                                              _ptr(row_ptr), _ptr(col), int(col.numel()), _ptr(energy),
                                              _ptr(forces)))
@@ -210,10 +236,7 @@ class Context:
     def md_step(self, system, pos, vel, forces, types, mass: float, dt: float, n_steps: int,
                 energy, kinetic):
         import torch
-        for t, dtp, n in ((pos, torch.float32, "pos"), (vel, torch.float32, "vel"),
-                          (forces, torch.float32, "forces"), (types, torch.int32, "types"),
-                          (energy, torch.float32, "energy"), (kinetic, torch.float32, "kinetic")):
-            _dev_check(t, dtp, n)
+        _check_md_arrays(system, pos, vel, forces, types, energy, kinetic)
         self._check(self._L.sn_md_step(self._h, C.byref(system_struct(system)), _ptr(pos), _ptr(vel),
                                        _ptr(forces), _ptr(types), float(mass), float(dt), int(n_steps),
                                        _ptr(energy), _ptr(kinetic)))
@@ -222,10 +245,7 @@ class Context:
                     temperature: float, friction: float, seed: int, step0: int, energy, kinetic):
         """BAOAB Langevin steps (see sn_md_langevin); friction in 1/fs."""
         import torch
-        for t, dtp, n in ((pos, torch.float32, "pos"), (vel, torch.float32, "vel"),
-                          (forces, torch.float32, "forces"), (types, torch.int32, "types"),
-                          (energy, torch.float32, "energy"), (kinetic, torch.float32, "kinetic")):
-            _dev_check(t, dtp, n)
+        _check_md_arrays(system, pos, vel, forces, types, energy, kinetic)
         self._check(self._L.sn_md_langevin(self._h, C.byref(system_struct(system)), _ptr(pos), _ptr(vel),
                                            _ptr(forces), _ptr(types), float(mass), float(dt), int(n_steps),
                                            float(temperature), float(friction), C.c_uint64(seed),
@@ -265,8 +285,9 @@ def build_neighbors_noalloc(system, r_cut: float, pos, row_ptr, col, stream=None
     CAPACITY)."""
     import torch
     L = load()
-    _dev_check(pos, torch.float32, "pos")
-    _dev_check(row_ptr, torch.int32, "row_ptr")
+    N = system.n_per_replica * system.n_replicas
+    _dev_check(pos, torch.float32, "pos", 3 * N)
+    _dev_check(row_ptr, torch.int32, "row_ptr", N + 1)
     _dev_check(col, torch.int32, "col")
     if stream is None:
         stream = torch.cuda.current_stream()

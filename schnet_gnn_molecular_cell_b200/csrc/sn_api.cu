@@ -156,7 +156,7 @@ sn_status ensure_nb(sn_ctx *ctx, const sn_system *s)
     if ((st = grow(ctx, ctx->cnt, sizeof(int32_t) * (N + 1)))) return st;
     if ((st = grow(ctx, ctx->cell_of, sizeof(int32_t) * N))) return st;
     if ((st = grow(ctx, ctx->cell_atoms, sizeof(int32_t) * N))) return st;
-    if ((st = grow(ctx, ctx->cell_cnt, sizeof(int32_t) * (ncell + 1)))) return st;
+    if ((st = grow(ctx, ctx->cell_cnt, sizeof(int32_t) * (ncell + 2)))) return st;
     if ((st = grow(ctx, ctx->cell_start, sizeof(int32_t) * (ncell + 1)))) return st;
     return SN_OK;
 }
@@ -186,7 +186,7 @@ sn::NbWork nb_work(sn_ctx *ctx)
     w.cell_cnt = (int32_t *)ctx->cell_cnt.p;
     w.cell_start = (int32_t *)ctx->cell_start.p;
     w.cell_atoms = (int32_t *)ctx->cell_atoms.p;
-    w.ncell_cap = (int64_t)(ctx->cell_cnt.bytes / sizeof(int32_t)) - 1;
+    w.ncell_cap = (int64_t)(ctx->cell_cnt.bytes / sizeof(int32_t)) - 2;
     return w;
 }
 
@@ -283,7 +283,8 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
     if (!(cfg->r_cut > 0.0f) || isinf(cfg->r_cut) || !(cfg->gamma > 0.0f) || NT < 1 || K < 2 || T < 1 || F < 2)
         return SN_ERR_INVALID_ARG;
     if (!(F == 64 || F == 128) || K > 64 || T > MAX_T) return SN_ERR_UNSUPPORTED;
-    if (cfg->precision != SN_PREC_FP32 && cfg->precision != SN_PREC_FP16 && cfg->precision != SN_PREC_TC32)
+    if (cfg->precision != SN_PREC_FP32 && cfg->precision != SN_PREC_FP16 && cfg->precision != SN_PREC_TC32 &&
+        cfg->precision != SN_PREC_FP16_CH)
         return SN_ERR_INVALID_ARG;
     if (cfg->precision != SN_PREC_FP32 && F != 128) return SN_ERR_UNSUPPORTED;
     const int H = F / 2;
@@ -342,6 +343,30 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
         }
     }
 
+    // Per-output-channel scales (SN_PREC_FP16_CH: the row's largest magnitude, 1 for a zero
+    // row; every other mode: 1): per block s1, s2, su1, su2 [F], then sr1 [F] (1 past H).
+    const bool per_channel = cfg->precision == SN_PREC_FP16_CH;
+    auto row_scales = [&](const float *W, int rows, int cols) {
+        size_t off = pk.take(F);
+        for (int r = 0; r < F; ++r) {
+            float m = 0.0f;
+            if (per_channel && r < rows)
+                for (int c = 0; c < cols; ++c) m = fmaxf(m, fabsf(W[(size_t)r * cols + c]));
+            pk.buf[off + r] = m > 0.0f ? m : 1.0f;
+        }
+        return off;
+    };
+    size_t o_scale[MAX_T][4];
+    for (int t = 0; t < T; ++t) {
+        const float *blk = weights_host + (int64_t)NT * F + t * per_block;
+        const float *W2 = blk + (int64_t)F * K + F, *U1 = W2 + (int64_t)F * F + F, *U2 = U1 + (int64_t)F * F + F;
+        o_scale[t][0] = row_scales(blk, F, K);
+        o_scale[t][1] = row_scales(W2, F, F);
+        o_scale[t][2] = row_scales(U1, F, F);
+        o_scale[t][3] = row_scales(U2, F, F);
+    }
+    const size_t o_sr1 = row_scales(weights_host + (int64_t)NT * F + T * per_block, H, F);
+
     // fp16 hi/lo copies of W1 and W2 in the tensor-core operand layout (per block: W1h W1l W2h W2l)
     std::vector<uint16_t> tcw;
     // per block: W1 hi, lo, W2 hi, lo, U1 hi, lo, U2 hi, lo; then R1 (padded to F rows) hi, lo
@@ -352,14 +377,15 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
             const float *blk = weights_host + (int64_t)NT * F + t * per_block;
             uint16_t *o = tcw.data() + per_tc * t;
             const float *W2 = blk + (int64_t)F * K + F, *U1 = W2 + (int64_t)F * F + F, *U2 = U1 + (int64_t)F * F + F;
-            sn::tc_pack_matrix(blk, F, K, KP, o, o + n_w1);
-            sn::tc_pack_matrix(W2, F, F, F, o + 2 * n_w1, o + 2 * n_w1 + n_w2);
-            sn::tc_pack_matrix(U1, F, F, F, o + 2 * n_w1 + 2 * n_w2, o + 2 * n_w1 + 3 * n_w2);
-            sn::tc_pack_matrix(U2, F, F, F, o + 2 * n_w1 + 4 * n_w2, o + 2 * n_w1 + 5 * n_w2);
+            const float *sc = pk.buf.data();
+            sn::tc_pack_matrix(blk, F, K, KP, sc + o_scale[t][0], o, o + n_w1);
+            sn::tc_pack_matrix(W2, F, F, F, sc + o_scale[t][1], o + 2 * n_w1, o + 2 * n_w1 + n_w2);
+            sn::tc_pack_matrix(U1, F, F, F, sc + o_scale[t][2], o + 2 * n_w1 + 2 * n_w2, o + 2 * n_w1 + 3 * n_w2);
+            sn::tc_pack_matrix(U2, F, F, F, sc + o_scale[t][3], o + 2 * n_w1 + 4 * n_w2, o + 2 * n_w1 + 5 * n_w2);
         }
         const float *R1 = weights_host + (int64_t)NT * F + T * per_block;
         uint16_t *o = tcw.data() + per_tc * T;
-        sn::tc_pack_matrix(R1, H, F, F, o, o + n_w2);   // rows H..F-1 stay zero
+        sn::tc_pack_matrix(R1, H, F, F, pk.buf.data() + o_sr1, o, o + n_w2);   // rows H..F-1 stay zero
     }
 
     cudaError_t e = cudaMalloc(&ctx->d_weights, sizeof(float) * pk.buf.size());
@@ -404,6 +430,10 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
         m.blk[t].c1 = W + o_blk[t][5];
         m.blk[t].U2 = W + o_blk[t][6];
         m.blk[t].c2 = W + o_blk[t][7];
+        m.blk[t].s1 = W + o_scale[t][0];
+        m.blk[t].s2 = W + o_scale[t][1];
+        m.blk[t].su1 = W + o_scale[t][2];
+        m.blk[t].su2 = W + o_scale[t][3];
         if (ctx->d_tcw) {
             const uint16_t *o = ctx->d_tcw + per_tc * t;
             m.blk[t].W1h = o;
@@ -420,6 +450,7 @@ sn_status sn_create(const sn_config *cfg, const float *weights_host, int64_t n_w
     m.ro.e1 = W + o_e1;
     m.ro.R2 = W + o_R2;
     m.ro.e2 = W + o_e2;
+    m.ro.sr1 = W + o_sr1;
     if (ctx->d_tcw) {
         m.ro.R1h = ctx->d_tcw + per_tc * T;
         m.ro.R1l = ctx->d_tcw + per_tc * T + n_w2;

@@ -625,6 +625,8 @@ EdgeTcArgs tc_args(const EdgeArgs &a, const BlockW &bw, int *d_err)
     t.W2l = bw.W2l;
     t.b1 = bw.b1;
     t.b2 = bw.b2;
+    t.s1 = bw.s1;
+    t.s2 = bw.s2;
     t.t = a.t;
     t.d_err = d_err;
     return t;
@@ -719,6 +721,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
         nt.e1 = m.ro.e1;
         nt.R2 = m.ro.R2;
         nt.e2 = m.ro.e2;
+        nt.sr1 = m.ro.sr1;
         nt.d_err = d_err;
         auto node_args = [&](int t) {
             NodeTcArgs a = nt;
@@ -729,6 +732,8 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
             a.U2l = m.blk[t].U2l;
             a.c1 = m.blk[t].c1;
             a.c2 = m.blk[t].c2;
+            a.su1 = m.blk[t].su1;
+            a.su2 = m.blk[t].su2;
             return a;
         };
         for (int t = 0; t < m.T; ++t) {

@@ -66,7 +66,10 @@ struct TcSmem {
     static constexpr uint32_t UVEC = DST + 4 * TE;      // float[TE][3]
     static constexpr uint32_t FV = UVEC + 12 * TE;      // float[TE][3]
     static constexpr uint32_t MASK = FV + 12 * TE;      // uint32[4]: row starts, empty-row flags
-    static constexpr uint32_t MBAR = MASK + 16;         // uint64
+    static constexpr uint32_t CD = MASK + 16;           // float2[TE]: C(d), dC/dd (fp16 backward)
+    static constexpr uint32_t TDST = CD + 8 * TE;       // int[TE]: type of the destination (block 0)
+    static constexpr uint32_t PDX = TDST + 4 * TE;      // float[4]: force scan, warp 0 -> warp 1
+    static constexpr uint32_t MBAR = PDX + 16;          // uint64
     static constexpr uint32_t REGION = (MBAR + 8 + 127) / 128 * 128;
     static constexpr uint32_t HOLD = GROUPS + NW * REGION;
     static constexpr uint32_t WMBAR = HOLD + 8;           // weight copies
@@ -90,14 +93,16 @@ struct EdgePos {
     float4 ri, rj;
     int tj, rs;   // type of the source (block 0), first edge of the destination's row
     int rsm;      // first edge of the row before the destination's (-1 for row 0)
+    int ti;       // type of the destination (block 0)
 };
 
+// (loads kept where they stand, so that the read-ahead by a tile really is ahead: see ld_keep)
 __device__ __forceinline__ EdgeIdx load_idx(const EdgeTcArgs &A, int e, int e1)
 {
     EdgeIdx x{0, 0};
     if (e < e1) {
-        x.i = __ldg(A.dst + e);
-        x.j = __ldg(A.col + e);
+        x.i = ldnc_keep(A.dst + e);
+        x.j = ldnc_keep(A.col + e);
     }
     return x;
 }
@@ -105,11 +110,12 @@ __device__ __forceinline__ EdgeIdx load_idx(const EdgeTcArgs &A, int e, int e1)
 __device__ __forceinline__ EdgePos load_pos(const EdgeTcArgs &A, EdgeIdx x)
 {
     EdgePos p;
-    p.ri = __ldg(A.pos4 + x.i);
-    p.rj = __ldg(A.pos4 + x.j);
-    p.tj = A.t == 0 ? __ldg(A.types + x.j) : 0;
-    p.rs = __ldg(A.row_ptr + x.i);
-    p.rsm = x.i > 0 ? __ldg(A.row_ptr + x.i - 1) : -1;
+    p.ri = ldnc_keep(A.pos4 + x.i);
+    p.rj = ldnc_keep(A.pos4 + x.j);
+    p.tj = A.t == 0 ? ldnc_keep(A.types + x.j) : 0;
+    p.rs = ldnc_keep(A.row_ptr + x.i);
+    p.rsm = x.i > 0 ? ldnc_keep(A.row_ptr + x.i - 1) : -1;
+    p.ti = A.t == 0 ? ldnc_keep(A.types + x.i) : 0;
     return p;
 }
 
@@ -133,7 +139,9 @@ __device__ __forceinline__ const float *x_row(const EdgeTcArgs &A, const float *
 // also the offsets of the source's feature rows used by the gathers (padding edges: 0).
 // SHARED (fp16, warp-specialised producer): part 0 alone forms d and C(d) and leaves them in
 // the stage (S::DF, S::CC) for the other parts, after a barrier over the 64 PARTS threads.
-template <class S, int KP, bool SPLIT, bool BWD, int PARTS = 2, bool SHARED = false>
+// STORE_CD (fp16 backward): part 0 also leaves C(d) and dC/dd of every edge in the stage
+// (S::CD, float2[TE]) for the dbar step, and the destination's type (S::TDST, int[TE], block 0).
+template <class S, int KP, bool SPLIT, bool BWD, int PARTS = 2, bool SHARED = false, bool STORE_CD = false>
 __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigned char *sm, unsigned char *R, int t,
                                               int ts, int ne, EdgeIdx x, const EdgePos &p)
 {
@@ -158,6 +166,7 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
         d = sqrt(dx * dx + dy * dy + dz * dz);
         if (half == 0) {
             sDst[n] = i;
+            if constexpr (STORE_CD) reinterpret_cast<int *>(R + S::TDST)[n] = p.ti;
             sDist[n] = (double)d;
             const real inv = (real)1 / d;
             sU[3 * n] = (float)(dx * inv);
@@ -169,6 +178,7 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
         }
     } else if (half == 0) {
         sDst[n] = -1;
+        if constexpr (STORE_CD) reinterpret_cast<int *>(R + S::TDST)[n] = 0;
         sDist[n] = 0.0;
     } else if (half == 1) {
         if (BWD) reinterpret_cast<int2 *>(sXo)[n] = make_int2(0, 0);
@@ -197,6 +207,15 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
         named_sync(5, 64 * PARTS);
         d_hi = reinterpret_cast<const float *>(R + S::DF)[n];
         C = reinterpret_cast<const float *>(R + S::CC)[n];
+        d_lo = 0.0f;
+    } else if constexpr (STORE_CD) {
+        static_assert(!SPLIT, "the stored envelope is for fp16 operands");
+        float sn, cs;
+        sincospif((float)d / A.basis.r_cut, &sn, &cs);
+        C = 0.5f * (cs + 1.0f);
+        if (half == 0)
+            reinterpret_cast<float2 *>(R + S::CD)[n] = make_float2(C, -0.5f * (float)M_PI / A.basis.r_cut * sn);
+        d_hi = (float)d;
         d_lo = 0.0f;
     } else {
         C = 0.5f * (cospif(SPLIT ? (float)((double)d / A.basis.r_cut_d) : (float)d / A.basis.r_cut) + 1.0f);
@@ -379,14 +398,14 @@ __device__ __forceinline__ bool mma_step(const Group &G, uint32_t &phase, int *d
 
 // s = ssp(a + b1) from TMEM columns [COL_A, COL_A + TE) into the activation tile
 template <bool SPLIT, int CH>
-__device__ __forceinline__ void ssp_to_tile(const Group &G, float b1f, unsigned char *Th, unsigned char *Tl)
+__device__ __forceinline__ void ssp_to_tile(const Group &G, float s1f, float b1f, unsigned char *Th, unsigned char *Tl)
 {
 #pragma unroll 1
     for (int c = 0; c < TE / CH; ++c) {
         float v[CH];
         tmem_ld<CH>(G.tm + G.lane + COL_A + CH * c, v);
 #pragma unroll
-        for (int q = 0; q < CH; ++q) v[q] = ssp_mode<SPLIT>(v[q] + b1f);
+        for (int q = 0; q < CH; ++q) v[q] = ssp_mode<SPLIT>(fmaf(v[q], s1f, b1f));
         store_tile_col<SPLIT, CH>(Th, Tl, G.t, CH * c, v);
     }
 }
@@ -402,7 +421,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
     const int f = G.t;
     if (!skip && G.i0 < G.i1) {
         const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
-        const float b1f = A.b1[f], b2f = A.b2[f];
+        const float b1f = A.b1[f], b2f = A.b2[f], s1f = A.s1[f], s2f = A.s2[f];
         const float *xbase = x_base(A, f);
         const int *sXo = reinterpret_cast<const int *>(G.R + S::XO);
         const int *sDst = reinterpret_cast<const int *>(G.R + S::DST);
@@ -429,7 +448,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
                         hacc = 0.0f;
                         cur = i;
                     }
-                    hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                    hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
                 }
             }
         };
@@ -444,7 +463,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
             if (more) nidx = load_idx(A, ts + TE + nf, e1);
             if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<S, KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
-            ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
+            ssp_to_tile<SPLIT, CH>(G, s1f, b1f, Th, Tl);
             if (more) npos = load_pos(A, nidx);
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
                 break;
@@ -480,7 +499,8 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
     const int f = G.t;
     if (!skip && G.i0 < G.i1) {
         const int e0 = A.row_ptr[G.i0], e1 = A.row_ptr[G.i1];
-        const float b1f = A.b1[f], b2f = A.b2[f];
+        const float b1f = A.b1[f], b2f = A.b2[f], s1f = A.s1[f], s2f = A.s2[f];
+        const float hs1 = 0.5f * s1f, hb1 = 0.5f * b1f;
         const float *xbase = x_base(A, f), *hbase = A.Hbar + f;
         const int2 *sOff = reinterpret_cast<const int2 *>(G.R + S::XO);
         const uint32_t *sMask = reinterpret_cast<const uint32_t *>(G.R + S::MASK);
@@ -492,7 +512,9 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         uint32_t phase = 0;
         bool ok = true;
         // Destination-row state: the running xbar sum of row cur, the row's own xbar, x_i and
-        // hbar_i, and the same values of row cur + 1 read ahead (the usual next row).
+        // hbar_i, and the same values of row cur + 1 read ahead (the usual next row).  x_i and
+        // hbar_i enter only wbar, which is W2's transposed operand: they carry W2's channel
+        // scale s2 (wbar s2 = x_j (hbar_i s2) + (x_i s2) hbar_j).
         int cur = -1, nrow = -1;
         float xbacc = 0.0f, xbold = 0.0f, xi_c = 0.0f, hi_c = 0.0f, nxb = 0.0f, nxi = 0.0f, nhi = 0.0f;
         auto next_row = [&](int i) {
@@ -501,18 +523,19 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
             cur = i;
             if (i == nrow) {
                 xbold = nxb;
-                xi_c = nxi;
-                hi_c = nhi;
+                xi_c = nxi * s2f;
+                hi_c = nhi * s2f;
             } else {
                 xbold = A.Xbar[(int64_t)i * FF + f];
-                xi_c = __ldg(x_row(A, xbase, i));
-                hi_c = __ldg(hbase + (int64_t)i * FF);
+                xi_c = __ldg(x_row(A, xbase, i)) * s2f;
+                hi_c = __ldg(hbase + (int64_t)i * FF) * s2f;
             }
             nrow = i + 1 < A.N ? i + 1 : -1;
-            if (nrow >= 0) {   // discarded unless row i + 1 is this group's next row
-                nxb = A.Xbar[(int64_t)nrow * FF + f];
-                nxi = __ldg(x_row(A, xbase, nrow));
-                nhi = __ldg(hbase + (int64_t)nrow * FF);
+            if (nrow >= 0) {   // discarded unless row i + 1 is this group's next row; the loads
+                               // stay here (ld_keep) and are scaled when the row starts
+                nxb = ld_keep(A.Xbar + (int64_t)nrow * FF + f);
+                nxi = ldnc_keep(x_row(A, xbase, nrow));
+                nhi = ldnc_keep(hbase + (int64_t)nrow * FF);
             }
         };
         // xbar_i += hbar_j (.) (w + b2) and the tile of wbar = x_j (.) hbar_i + x_i (.) hbar_j over
@@ -533,7 +556,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
             if (FULL && m == 0) {
 #pragma unroll
                 for (int q = 0; q < CH; ++q) {
-                    xbacc = fmaf(hb[q], w[q] + b2f, xbacc);
+                    xbacc = fmaf(hb[q], fmaf(w[q], s2f, b2f), xbacc);
                     xj[q] = xj[q] * hi_c + xi_c * hb[q];
                 }
             } else {
@@ -542,7 +565,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                     const int n = CH * c + q;
                     if (FULL || n < ne) {
                         if ((m >> q) & 1u) next_row(sDst[n]);
-                        xbacc = fmaf(hb[q], w[q] + b2f, xbacc);
+                        xbacc = fmaf(hb[q], fmaf(w[q], s2f, b2f), xbacc);
                         xj[q] = xj[q] * hi_c + xi_c * hb[q];
                     } else {
                         xj[q] = 0.0f;
@@ -556,12 +579,12 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         EdgePos npos = load_pos(A, nidx);
         for (int ts = e0; ts < e1 && ok; ts += TE) {
             const int ne = min(TE, e1 - ts);
-            tile_prologue<S, KP, SPLIT, true>(A, sm, G.R, f, ts, ne, nidx, npos);
+            tile_prologue<S, KP, SPLIT, true, 2, false, !SPLIT>(A, sm, G.R, f, ts, ne, nidx, npos);
             const bool more = ts + TE < e1;
             if (more) nidx = load_idx(A, ts + TE + nf, e1);
             if (ts == e0 && !(ok = wait_weights<KP, SPLIT, NW>(G, sm, A.d_err))) break;
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma1<S, KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
-            ssp_to_tile<SPLIT, CH>(G, b1f, Th, Tl);
+            ssp_to_tile<SPLIT, CH>(G, s1f, b1f, Th, Tl);
             if (more) npos = load_pos(A, nidx);
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
                 break;
@@ -573,14 +596,14 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
             }
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, true>(sm, G.R, G.tm + COL_W); })))
                 break;
-            // abar = sbar (.) sigma(a + b1)
+            // abar = sbar (.) sigma(a s1 + b1), times W1's channel scale s1 (W1's transposed operand)
 #pragma unroll 1
             for (int c = 0; c < TE / CH; ++c) {
                 float sb[CH], a[CH];
                 tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, sb);
                 tmem_ld<CH>(G.tm + G.lane + COL_A + CH * c, a);
 #pragma unroll
-                for (int q = 0; q < CH; ++q) sb[q] *= sigmoid_mode<SPLIT>(a[q] + b1f);
+                for (int q = 0; q < CH; ++q) sb[q] *= sigmoid_scaled<SPLIT>(a[q], s1f, b1f, hs1, hb1);
                 store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, sb);
             }
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma4<S, KP, SPLIT>(sm, G.R, G.tm + COL_A); }))) break;
@@ -592,9 +615,16 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 const int n = 16 * (f >> 5) + 8 * (l & 1) + (l >> 2);
                 const bool mine = n < ne;
                 const double d = mine ? sDist[n] : 0.0;
-                const float ratio = (float)(d / A.basis.r_cut_d);
-                const float C = 0.5f * (cospif(ratio) + 1.0f);
-                const float dC = -0.5f * (float)M_PI / A.basis.r_cut * sinpif(ratio);
+                float C, dC;
+                if constexpr (SPLIT) {
+                    const float ratio = (float)(d / A.basis.r_cut_d);
+                    C = 0.5f * (cospif(ratio) + 1.0f);
+                    dC = -0.5f * (float)M_PI / A.basis.r_cut * sinpif(ratio);
+                } else {   // formed once per edge by the prologue
+                    const float2 cd = mine ? reinterpret_cast<const float2 *>(G.R + S::CD)[n] : make_float2(0.0f, 0.0f);
+                    C = cd.x;
+                    dC = cd.y;
+                }
                 const float cc = -2.0f * A.basis.gamma * C, g2 = -A.basis.gamma * LOG2EF;
                 const float d_hi = (float)d, d_lo = (float)(d - (double)d_hi);
                 const float *mh = reinterpret_cast<const float *>(sm + S::MUH) + par;
@@ -621,18 +651,51 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
             }
             tc_fence_before();
             wg_sync(G.g);
-            // one thread per row segment of the tile sums its edges' forces in edge order
-            if (f < ne && (f == 0 || sDst[f] != sDst[f - 1])) {
-                const int row = sDst[f];
-                float fx = 0.0f, fy = 0.0f, fz = 0.0f;
-                for (int n = f; n < ne && sDst[n] == row; ++n) {
-                    fx += sFv[3 * n];
-                    fy += sFv[3 * n + 1];
-                    fz += sFv[3 * n + 2];
+            if (f < TE) {
+                // the tile's edge forces summed per destination row: segmented scan over edge
+                // n = f in the group's first two warps (the second warp's leading segment adds the
+                // first warp's last partial sum); the last edge of each segment adds the row's
+                // sum to the forces with a reduction that returns nothing.  All additions to a
+                // row come from this group, tile after tile, separated by its barriers, so their
+                // order is fixed.
+                const int lane = f & 31;
+                const bool valid = f < ne;
+                const int row = valid ? sDst[f] : -1;
+                float fx = valid ? sFv[3 * f] : 0.0f, fy = valid ? sFv[3 * f + 1] : 0.0f,
+                      fz = valid ? sFv[3 * f + 2] : 0.0f;
+                int fl = valid && (f == 0 || sDst[f - 1] != row);
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float px = __shfl_up_sync(0xffffffffu, fx, o);
+                    const float py = __shfl_up_sync(0xffffffffu, fy, o);
+                    const float pz = __shfl_up_sync(0xffffffffu, fz, o);
+                    const int pf = __shfl_up_sync(0xffffffffu, fl, o);
+                    if (lane >= o) {
+                        if (!fl) {
+                            fx += px;
+                            fy += py;
+                            fz += pz;
+                        }
+                        fl |= pf;
+                    }
                 }
-                A.forces[(int64_t)row * 3] += fx;
-                A.forces[(int64_t)row * 3 + 1] += fy;
-                A.forces[(int64_t)row * 3 + 2] += fz;
+                float *sPX = reinterpret_cast<float *>(G.R + S::PDX);
+                if (f == 31) {
+                    sPX[0] = fx;
+                    sPX[1] = fy;
+                    sPX[2] = fz;
+                }
+                named_sync(5 + G.g, TE);
+                if (f >= 32 && !fl) {
+                    fx += sPX[0];
+                    fy += sPX[1];
+                    fz += sPX[2];
+                }
+                if (valid && (f == ne - 1 || sDst[f + 1] != row)) {
+                    atomicAdd(A.forces + (int64_t)row * 3, fx);
+                    atomicAdd(A.forces + (int64_t)row * 3 + 1, fy);
+                    atomicAdd(A.forces + (int64_t)row * 3 + 2, fz);
+                }
             }
             wg_sync(G.g);
         }
@@ -860,7 +923,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
         } else if (warp < 16) {
             // S: s = ssp(a + b1) into the stage's activation tile, columns [32 sg, 32 sg + 32)
             const int f = (threadIdx.x - WS_P) % WGT, sg = (threadIdx.x - WS_P) / WGT;
-            const float b1f = A.b1[f];
+            const float b1f = A.b1[f], s1f = A.s1[f];
             const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
             for (int k = 0; k < nt; ++k) {
                 const int s = k % NSTG;
@@ -872,7 +935,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                     float v[CH];
                     tmem_ld<CH>(tmem + lanes + 64 * s + CH * c, v);
 #pragma unroll
-                    for (int q = 0; q < CH; ++q) v[q] = ssp_mode<SPLIT>(v[q] + b1f);
+                    for (int q = 0; q < CH; ++q) v[q] = ssp_mode<SPLIT>(fmaf(v[q], s1f, b1f));
                     store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, v);
                 }
                 tc_fence_before();
@@ -883,7 +946,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
             // E: h_i += x_src (.) (w + b2); a row is written when the next one starts (rows in
             // between, and after the last edge, have no edges and receive zero)
             const int f = threadIdx.x - WS_P - WS_S;
-            const float b2f = A.b2[f];
+            const float b2f = A.b2[f], s2f = A.s2[f];
             const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
             int cur = r0;
             float hacc = 0.0f;
@@ -910,7 +973,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                     const uint32_t m = (uint32_t)(starts >> (CH * c)) & (CH >= 32 ? 0xffffffffu : (1u << (CH & 31)) - 1u);
                     if (FAST && m == 0) {   // the chunk continues the current row
 #pragma unroll
-                        for (int q = 0; q < CH; ++q) hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                        for (int q = 0; q < CH; ++q) hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
                         return;
                     }
                     if (FAST && (m & (m - 1u)) == 0) {
@@ -921,7 +984,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
 #pragma unroll
                         for (int q = 0; q < CH; ++q) {
                             const bool before = q < p;
-                            const float t0 = fmaf(xs[q], v[q] + b2f, before ? a0 : b0);
+                            const float t0 = fmaf(xs[q], fmaf(v[q], s2f, b2f), before ? a0 : b0);
                             a0 = before ? t0 : a0;
                             b0 = before ? b0 : t0;
                         }
@@ -941,7 +1004,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                             store_if(A.H + (int64_t)cur * FF + f, hacc, st);
                             hacc = st ? 0.0f : hacc;
                             cur = st ? dst[q] : cur;
-                            hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                            hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
                         } else if (n < ne) {
                             if (st) {   // first edge of row dst[q]; rows in between have no edges
                                 store_if(A.H + (int64_t)cur * FF + f, hacc, true);
@@ -949,7 +1012,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                                 hacc = 0.0f;
                                 cur = dst[q];
                             }
-                            hacc = fmaf(xs[q], v[q] + b2f, hacc);
+                            hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
                         }
                     }
                 };
@@ -1032,13 +1095,15 @@ cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backwar
 
 // Host: one weight matrix W[rows][cols] (fp32, row-major) into the core-matrix layout used by
 // the kernels (element (r, c) at half index ((r%8)*16 + (r/8)*SBO + (c%8)*2 + (c/8)*128)/2,
-// SBO = (cols_pad/8)*128 bytes, columns cols..cols_pad-1 zero), as fp16 hi and lo = fp16(w - hi).
-void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, uint16_t *hi, uint16_t *lo)
+// SBO = (cols_pad/8)*128 bytes, columns cols..cols_pad-1 zero), as fp16 hi and lo = fp16(w - hi)
+// of w = W[r][c] / row_scale[r] (the division in fp32).
+void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, const float *row_scale, uint16_t *hi,
+                    uint16_t *lo)
 {
     const size_t sbo = (size_t)(cols_pad / 8) * 128;
     for (int r = 0; r < rows; ++r)
         for (int c = 0; c < cols_pad; ++c) {
-            const float w = c < cols ? W[(size_t)r * cols + c] : 0.0f;
+            const float w = c < cols ? W[(size_t)r * cols + c] / row_scale[r] : 0.0f;
             const __half h = __float2half_rn(w);
             const __half l = __float2half_rn(w - __half2float(h));
             const size_t byte = (size_t)(r % 8) * 16 + (size_t)(r / 8) * sbo + (size_t)(c % 8) * 2 + (size_t)(c / 8) * 128;

@@ -64,6 +64,9 @@ struct BlockW {
     // tensor-core precisions: W1, W2, U1, U2 as fp16 hi / lo in the core-matrix layout of
     // sn_ef_tc.cu (lo = fp16(w - hi), used by the split mode)
     const void *W1h, *W1l, *W2h, *W2l, *U1h, *U1l, *U2h, *U2l;
+    // per-output-channel scales of W1, W2, U1, U2 ([F] each; all 1 except SN_PREC_FP16_CH):
+    // the fp16 matrices hold W[o][:] / s[o]
+    const float *s1, *s2, *su1, *su2;
 };
 
 struct ReadoutW {
@@ -72,6 +75,7 @@ struct ReadoutW {
     const float *R2;   // [H]
     const float *e2;   // [1]
     const void *R1h, *R1l;   // tensor-core precisions: R1 padded to 128 rows, fp16 hi / lo
+    const float *sr1;        // [128] per-output-channel scales of R1 (1 past H)
 };
 
 struct Geometry {
@@ -102,7 +106,7 @@ struct NbWork {
     float4 *pos4;      // [N]
     int32_t *cnt;      // [N + 1]
     int32_t *cell_of;  // [N]
-    int32_t *cell_cnt; // [ncell + 1]
+    int32_t *cell_cnt; // [ncell + 2]: counts / cursors, then (last entry) the stencil flag
     int32_t *cell_start; // [ncell + 1]
     int32_t *cell_atoms; // [N]
     int64_t ncell_cap;
@@ -161,13 +165,15 @@ struct EdgeTcArgs {
     Basis basis;
     const void *W1h, *W1l, *W2h, *W2l;
     const float *b1, *b2;
+    const float *s1, *s2;  // [F] output-channel scales of W1 and W2
     int t;
     int *d_err;
 };
 
 cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s);
 int tc_groups_per_cta(bool split);   // independent row ranges per CTA of the tensor-core edge kernels
-void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, uint16_t *hi, uint16_t *lo);
+void tc_pack_matrix(const float *W, int rows, int cols, int cols_pad, const float *row_scale, uint16_t *hi,
+                    uint16_t *lo);
 
 // Arguments of the tensor-core node kernels (F = 128).
 struct NodeTcArgs {
@@ -184,6 +190,7 @@ struct NodeTcArgs {
     int t;
     const void *U1h, *U1l, *U2h, *U2l, *R1h, *R1l;
     const float *c1, *c2, *e1, *R2, *e2;
+    const float *su1, *su2, *sr1;   // output-channel scales of U1, U2 ([F]) and R1 ([128])
     int *d_err;
 };
 

@@ -11,7 +11,13 @@
 //   * open boundaries (or a box too small for a 3x3x3 cell stencil): all pairs of a replica,
 //     positions staged through shared memory in tiles of 128; sources come out ascending;
 //   * periodic boxes with >= 3 cells per axis: cell list (cell side >= r_cut * 1.0001), then
-//     each row is sorted by source.
+//     each row is sorted by source.  Atoms are binned by their coordinates wrapped into the
+//     box in double precision.  The fp32 test on raw coordinates can accept a pair whose
+//     exact separation exceeds r_cut by its rounding error, which grows with |x|; while every
+//     |coordinate| stays below a bound derived from the cell margin (side - r_cut) that error
+//     is smaller than the margin and the 27-cell stencil holds every accepted pair.  An atom
+//     beyond the bound raises a flag in the cell workspace and both passes then test all
+//     pairs of each replica instead (same list, slower).
 // Both run a count pass, an exclusive scan into row_ptr, and a fill pass.
 #include <cuda_runtime.h>
 #include <math.h>
@@ -103,28 +109,35 @@ __global__ void __launch_bounds__(256) k_pairs(const float4 *__restrict__ pos4, 
 // -------------------------------------------------------------------- cell list (periodic)
 struct CellGrid {
     int nc[3];
-    float side[3];
+    double side[3];
     int64_t per_rep;
+    int n_per;
+    float x_safe;     // |coordinate| bound of the cell stencil (see file header)
+    int32_t *flag;    // set when an atom exceeds x_safe (cleared with the cell counters)
 };
 
-__device__ __forceinline__ int cell_coord(float x, float L, float side, int n)
+// cell index along one axis of the coordinate wrapped into [0, L) in double (x is exact in
+// double; the wrap and the division add ~1e-16 relative)
+__device__ __forceinline__ int cell_coord(float x, float L, double side, int n)
 {
-    float w = x - L * floorf(x / L);      // wrapped into [0, L] (L only through rounding)
-    int c = (int)floorf(w / side);
+    const double xd = (double)x, Ld = (double)L;
+    const double w = xd - Ld * floor(xd / Ld);
+    const int c = (int)floor(w / side);
     return c < 0 ? 0 : (c >= n ? n - 1 : c);
 }
 
-__global__ void k_cell_assign(const float4 *__restrict__ pos4, int64_t N, int n_per, Geometry g, CellGrid cg,
+__global__ void k_cell_assign(const float4 *__restrict__ pos4, int64_t N, Geometry g, CellGrid cg,
                               int32_t *__restrict__ cell_of, int32_t *__restrict__ cell_cnt,
                               const int *__restrict__ d_err)
 {
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= N || (*((volatile const int *)d_err) & ERRBIT_NONFINITE)) return;
     float4 p = pos4[i];
+    if (fmaxf(fabsf(p.x), fmaxf(fabsf(p.y), fabsf(p.z))) > cg.x_safe) *cg.flag = 1;
     int cx = cell_coord(p.x, g.box[0], cg.side[0], cg.nc[0]);
     int cy = cell_coord(p.y, g.box[1], cg.side[1], cg.nc[1]);
     int cz = cell_coord(p.z, g.box[2], cg.side[2], cg.nc[2]);
-    int64_t c = (i / n_per) * cg.per_rep + ((int64_t)cx * cg.nc[1] + cy) * cg.nc[2] + cz;
+    int64_t c = (i / cg.n_per) * cg.per_rep + ((int64_t)cx * cg.nc[1] + cy) * cg.nc[2] + cz;
     cell_of[i] = (int32_t)c;
     atomicAdd(&cell_cnt[c], 1);
 }
@@ -163,6 +176,22 @@ __global__ void __launch_bounds__(BT) k_cell_pairs(const float4 *__restrict__ po
     int32_t n = 0;
     const int32_t w0 = FILL ? row_ptr[i] : 0;
     bool degenerate = false;
+    if (*((volatile const int32_t *)cg.flag)) {
+        // a coordinate beyond the stencil's bound: every source of the replica, ascending
+        const int64_t b0 = i / cg.n_per * cg.n_per;
+        for (int64_t j = b0; j < b0 + cg.n_per; ++j) {
+            if (j == i) continue;
+            const float r2 = pair_r2(pi, pos4[j], g);
+            if (r2 < rc2) {
+                if (FILL) col[w0 + n] = (int32_t)j;
+                ++n;
+                degenerate |= (r2 == 0.0f);
+            }
+        }
+        if (FILL && degenerate) atomicOr(d_err, ERRBIT_DEGENERATE);
+        if (!FILL) cnt[i] = n;
+        return;
+    }
     for (int ox = -1; ox <= 1; ++ox)
         for (int oy = -1; oy <= 1; ++oy)
             for (int oz = -1; oz <= 1; ++oz) {
@@ -393,16 +422,26 @@ cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *po
     const bool cells = use_cells(sys, r_cut, nc);
     CellGrid cg{};
     if (cells) {
+        double margin = 1e300, Lmax = 0.0;
         for (int a = 0; a < 3; ++a) {
             cg.nc[a] = nc[a];
-            cg.side[a] = sys.box[a] / (float)nc[a];
+            cg.side[a] = (double)sys.box[a] / (double)nc[a];
+            margin = fmin(margin, cg.side[a] - (double)r_cut);
+            Lmax = fmax(Lmax, (double)sys.box[a]);
         }
+        // Per axis the fp32 test's separation is within 2^-22 |x|max + 2^-24 L of the exact
+        // one (rounding of x_j - x_i, of L * rint(.) and of their difference), the distance
+        // within sqrt(3) times that plus 2^-22 r_cut.  Half the margin is allowed for it.
+        const double slack = 0.5 * margin / sqrt(3.0) - ldexp(Lmax, -24) - ldexp((double)r_cut, -22) / sqrt(3.0);
+        cg.x_safe = slack > 0.0 ? (float)ldexp(slack, 22) : 0.0f;
         cg.per_rep = (int64_t)nc[0] * nc[1] * nc[2];
+        cg.n_per = sys.n_per_replica;
         const int64_t ncell = cg.per_rep * sys.n_replicas;
         if (ncell > w.ncell_cap) return cudaErrorInvalidValue;
-        if ((e = cudaMemsetAsync(w.cell_cnt, 0, sizeof(int32_t) * (ncell + 1), s))) return e;
+        cg.flag = w.cell_cnt + ncell + 1;
+        if ((e = cudaMemsetAsync(w.cell_cnt, 0, sizeof(int32_t) * (ncell + 2), s))) return e;
         trace_begin(tr, KK_CELLS, s);
-        k_cell_assign<<<blocks_for(N, 256), 256, 0, s>>>(pos4, N, sys.n_per_replica, g, cg, w.cell_of, w.cell_cnt, d_err);
+        k_cell_assign<<<blocks_for(N, 256), 256, 0, s>>>(pos4, N, g, cg, w.cell_of, w.cell_cnt, d_err);
         k_scan<<<1, 1024, 0, s>>>(w.cell_cnt, w.cell_start, ncell, d_err);
         // cursor = cell_start (reuse cell_cnt as the cursor array)
         k_copy_i32<<<blocks_for(ncell, 256), 256, 0, s>>>(w.cell_start, w.cell_cnt, ncell);

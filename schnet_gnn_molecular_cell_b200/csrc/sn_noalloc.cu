@@ -11,15 +11,12 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
-#include <mutex>
-
 #include "sn_internal.cuh"
 
 namespace {
 
 constexpr int64_t kMaxAtoms = SN_NOALLOC_MAX_ATOMS;
 constexpr int64_t kMaxCells = SN_NOALLOC_MAX_CELLS;
-constexpr int kMaxDevices = 64;
 
 constexpr size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -28,34 +25,25 @@ constexpr size_t kOffPos4 = 0;                                                  
 constexpr size_t kOffCnt = align256(kOffPos4 + sizeof(float4) * kMaxAtoms);     // int32 [kMaxAtoms + 1]
 constexpr size_t kOffCellOf = align256(kOffCnt + sizeof(int32_t) * (kMaxAtoms + 1));
 constexpr size_t kOffCellAtoms = align256(kOffCellOf + sizeof(int32_t) * kMaxAtoms);
-constexpr size_t kOffCellCnt = align256(kOffCellAtoms + sizeof(int32_t) * kMaxAtoms);   // [kMaxCells + 1]
-constexpr size_t kOffCellStart = align256(kOffCellCnt + sizeof(int32_t) * (kMaxCells + 1));
+constexpr size_t kOffCellCnt = align256(kOffCellAtoms + sizeof(int32_t) * kMaxAtoms);   // [kMaxCells + 2]
+constexpr size_t kOffCellStart = align256(kOffCellCnt + sizeof(int32_t) * (kMaxCells + 2));
 constexpr size_t kOffErr = align256(kOffCellStart + sizeof(int32_t) * (kMaxCells + 1)); // int32 error bits
 constexpr size_t kScratchBytes = align256(kOffErr + sizeof(int32_t));
 
 static __device__ __align__(256) unsigned char g_nb_scratch[kScratchBytes];
 
-std::mutex g_mutex;
-void *g_scratch_addr[kMaxDevices] = {};
-
 // Device address of g_nb_scratch on the current device.  In host code the symbol is only a
-// host-side stand-in; the address a kernel may use comes from cudaGetSymbolAddress, looked
-// up once per device with that device current.
+// host-side stand-in; the address a kernel may use comes from cudaGetSymbolAddress with that
+// device current.  It is looked up on every call (a host-side table lookup): a cached address
+// would go stale when cudaDeviceReset recreates the device's context and module.
 sn_status scratch_on_current_device(unsigned char **out)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return SN_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return SN_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_nb_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return SN_ERR_CUDA;
-        }
-        g_scratch_addr[dev] = p;
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_nb_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return SN_ERR_CUDA;
     }
-    *out = static_cast<unsigned char *>(g_scratch_addr[dev]);
+    *out = static_cast<unsigned char *>(p);
     return SN_OK;
 }
 

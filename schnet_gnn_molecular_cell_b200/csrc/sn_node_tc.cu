@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
     const uint32_t wmbar = smem_u32(sm + S::WMBAR);
     const int64_t n_tiles = (A.N + TA - 1) / TA;
     if (!skip) {
-        const float c1f = A.c1[f], c2f = A.c2[f];
+        const float c1f = A.c1[f], c2f = A.c2[f], su1f = A.su1[f], su2f = A.su2[f];
         unsigned char *T = sm + S::T;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const int64_t a = a0 + 32 * c + q;
-                    v[q] += c1f;
+                    v[q] = fmaf(v[q], su1f, c1f);
                     if (a < A.N) A.P[((int64_t)A.t * A.N + a) * FF + f] = v[q];
                     v[q] = ssp_fast(v[q]);
                 }
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const int64_t a = a0 + 32 * c + q;
-                    if (a < A.N) A.X[((int64_t)A.t * A.N + a) * FF + f] = xr[q] + v[q] + c2f;
+                    if (a < A.N) A.X[((int64_t)A.t * A.N + a) * FF + f] = fmaf(v[q], su2f, xr[q]) + c2f;
                 }
             }
             tc_fence_before();
@@ -215,6 +215,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_readout_tc(NodeTcArgs A)
     const int H = FF / 2;
     if (!skip) {
         const float e1k = f < H ? A.e1[f] : 0.0f, r2k = f < H ? A.R2[f] : 0.0f, e2 = A.e2[0];
+        const float sr1k = A.sr1[f], r2s = r2k * sr1k;   // R1's channel scale (1 past H)
         unsigned char *T = sm + S::T;
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
@@ -225,9 +226,9 @@ __global__ void __launch_bounds__(NT, 1) k_node_readout_tc(NodeTcArgs A)
                 tmem_ld32(tmem + lane + 32 * c, v);
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
-                    const float o = v[q] + e1k;
+                    const float o = fmaf(v[q], sr1k, e1k);
                     if (f < H) sPr[f * TA + 32 * c + q] = r2k * ssp_fast(o);
-                    v[q] = f < H ? r2k * sigmoid_fast(o) : 0.0f;
+                    v[q] = f < H ? r2s * sigmoid_fast(o) : 0.0f;   // R1's transposed operand
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
@@ -276,9 +277,11 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
     const int64_t n_tiles = (A.N + TA - 1) / TA;
     if (!skip) {
         unsigned char *T = sm + S::T;
+        // the operands of U2^T and U1^T carry the channel scales of U2 and U1
+        const float su1f = A.su1[f], su2f = A.su2[f];
         for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
-            tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.Xbar[a * FF + f]; });
+            tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.Xbar[a * FF + f] * su2f; });
             if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar)) break;
             {
                 float v[32];
@@ -287,7 +290,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
                 for (int q = 0; q < 32; ++q) {
                     const int64_t a = a0 + 32 * c + q;
                     const float p = a < A.N ? A.P[((int64_t)A.t * A.N + a) * FF + f] : 0.0f;
-                    v[q] *= sigmoid_fast(p);
+                    v[q] *= su1f * sigmoid_fast(p);
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }

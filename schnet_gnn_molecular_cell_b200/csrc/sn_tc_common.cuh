@@ -102,14 +102,17 @@ static __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(mbar), "r"(count) : "memory");
 }
 
+// Wait for a barrier phase, suspending the thread (it issues nothing meanwhile) until the phase
+// completes or about 0.2 ms have passed; false in the latter case.  Callers loop on it with
+// their own time bound.
 static __device__ __forceinline__ uint32_t mbar_try_wait(uint32_t mbar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(mbar), "r"(parity)
+        : "r"(mbar), "r"(parity), "r"(200000u)
         : "memory");
     return ok;
 }
@@ -177,6 +180,29 @@ static __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Two 16-column loads (this lane's columns at ta and at tb) completed by one wait.
+static __device__ __forceinline__ void tmem_ld16_pair(uint32_t ta, uint32_t tb, float (&a)[16], float (&b)[16])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31}, [%33];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(ta), "r"(tb)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        a[i] = __uint_as_float(r[i]);
+        b[i] = __uint_as_float(r[16 + i]);
+    }
 }
 
 template <int CH>
@@ -311,6 +337,34 @@ static __device__ __forceinline__ bool wait_mma_cta(uint32_t mbar, uint32_t &pha
 }
 
 
+// Loads issued where they stand: the compiler may move a plain load down to its first use,
+// which undoes a read-ahead; volatile asm keeps its place among the barrier operations
+// around it.  ".nc" for data that no thread writes during the kernel.
+static __device__ __forceinline__ float ld_keep(const float *p)
+{
+    float v;
+    asm volatile("ld.global.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
+static __device__ __forceinline__ float ldnc_keep(const float *p)
+{
+    float v;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+static __device__ __forceinline__ int ldnc_keep(const int *p)
+{
+    int v;
+    asm volatile("ld.global.nc.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+static __device__ __forceinline__ float4 ldnc_keep(const float4 *p)
+{
+    float4 v;
+    asm volatile("ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+    return v;
+}
+
 // Predicated global store (no branch); all stores of a value stream go through it so that
 // they keep their program order.
 static __device__ __forceinline__ void store_if(float *p, float v, bool c)
@@ -378,6 +432,16 @@ template <bool SPLIT>
 static __device__ __forceinline__ float sigmoid_mode(float x)
 {
     return SPLIT ? sigmoid_fast(x) : sigmoid16(x);
+}
+
+// s * sigma(v s + b) for a TMEM accumulator v of an output channel with scale s and bias b
+// (hs = s / 2, hb = b / 2): the scale of the channel carried into the operand of a transposed
+// product.  With s = 1 the value equals sigma_mode(v + b) exactly.
+template <bool SPLIT>
+static __device__ __forceinline__ float sigmoid_scaled(float v, float s, float b, float hs, float hb)
+{
+    if (SPLIT) return s * sigmoid_fast(fmaf(v, s, b));
+    return fmaf(hs, tanh_approx(fmaf(v, hs, hb)), hs);
 }
 
 }  // namespace tc

@@ -40,3 +40,17 @@ def test_create_rejects_bad_arguments_without_touching_the_gpu():
     bad = binding.Config(96, 50, 3, 20, 12.0, 10.0, 0)     # F = 96 is not built
     assert L.sn_create(ctypes.byref(bad), w.ctypes.data, 10, None, ctypes.byref(h)) == binding.Status.UNSUPPORTED
     assert h.value is None
+
+
+def test_every_status_of_the_header_has_a_binding_member():
+    # the binding turns every status the library can return into a Status member: an
+    # enumerator missing on the Python side would raise ValueError instead of SNError
+    text = (ROOT / "include" / "sn.h").read_text()
+    block = text[text.index("typedef enum {"):text.index("} sn_status;")]
+    block = re.sub(r"/\*.*?\*/", "", block, flags=re.S)
+    pairs = re.findall(r"\b(SN_(?:OK|ERR_[A-Z_]+))\s*=\s*(\d+)", block)
+    assert len(pairs) >= 9
+    for name, value in pairs:
+        short = name[len("SN_ERR_"):] if name.startswith("SN_ERR_") else "OK"
+        assert binding.Status[short] == int(value), name
+        assert isinstance(binding.SNError(int(value), "x").status, binding.Status)

@@ -179,3 +179,78 @@ def test_langevin_thermalises(dev):
     ctx.sync()
     ratio = np.mean(ke) / (1.5 * 64 * synth.KB * 300.0)
     assert abs(ratio - 1.0) < 0.05, ratio
+
+
+# ------------------------------------------------------------------ tensor-core precisions
+_ORACLE_TRAJ = {}
+
+
+def _oracle_traj(oracle, cfg, integrator, steps):
+    """The oracle's double-precision trajectory from the seeded start (cached: both tensor
+    modes compare against the same one)."""
+    key = (cfg, integrator, steps)
+    if key not in _ORACLE_TRAJ:
+        w = synth.make_workload(cfg)
+        s = w.system
+        v0 = synth.maxwell_boltzmann(s.n_per_replica, s.n_replicas, 12.0, 300.0, seed=4000 + cfg)
+        if integrator == "vv":
+            p, v, f, epot, ekin, _ = oracle.md_vv(w.model, w.weights, s, w.pos, v0, w.types, 12.0, 2.0, steps)
+        else:
+            p, v, f, epot, ekin = oracle.md_langevin(w.model, w.weights, s, w.pos, v0, w.types, 12.0, 4.0, steps,
+                                                     300.0, 0.01, seed=77)
+        _ORACLE_TRAJ[key] = (w, v0, p, v, f, ekin[-1])
+    return _ORACLE_TRAJ[key]
+
+
+@pytest.mark.parametrize("integrator", ["vv", "langevin"])
+@pytest.mark.parametrize("precision", [1, 2], ids=["fp16", "tc32"])
+@pytest.mark.parametrize("cfg", [2, 4])
+def test_md_tensor_modes_match_oracle(oracle, dev, cfg, precision, integrator):
+    """The benchmarked MD step in the tensor-core precisions against the oracle's trajectory
+    (velocity Verlet at 2 fs as the benchmark runs it; BAOAB Langevin at 4 fs with the
+    oracle's noise).  Trajectory: the deviation allowed on top of fp32 storage (as in
+    test_md_matches_oracle) is what the mode's force tolerance can cause over the run,
+    |dv| <= n dt kappa/m tol(F) and |dx| <= n^2 dt^2 kappa/m tol(F), tol(F) the mode's
+    per-component force bound (5e-3 |F| + 5e-3 RMS(F) for fp16; the fp32 bound for tc32).
+    Then energy and forces at the GPU's own final positions against the oracle at those
+    positions, at the mode's tolerance."""
+    from schnet_gnn_molecular_cell_b200 import Context
+    from tests.test_gpu_parity import assert_close
+    from tests.test_gpu_tensor import assert_close16
+    steps = 3
+    w, v0, p_o, v_o, f_o, ekin_o = _oracle_traj(oracle, cfg, integrator, steps)
+    s = w.system
+    ctx = Context(w.model, w.weights, precision=precision)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.from_numpy(v0.copy()).to(dev)
+    types = torch.from_numpy(w.types).to(dev)
+    rp, cl = ctx.neighbors(s, pos)
+    _, forces = ctx.energy_forces(s, pos, types, rp, cl)
+    forces = forces.clone()
+    energy = torch.empty(s.n_replicas, device=dev)
+    kin = torch.empty(s.n_replicas, device=dev)
+    if integrator == "vv":
+        dt = 2.0
+        ctx.md_step(s, pos, vel, forces, types, 12.0, dt, steps, energy, kin)
+    else:
+        dt = 4.0
+        ctx.md_langevin(s, pos, vel, forces, types, 12.0, dt, steps, 300.0, 0.01, 77, 0, energy, kin)
+    ctx.sync()
+    if precision == 1:
+        f_tol = 5e-3 * np.abs(f_o) + 5e-3 * np.sqrt(np.mean(f_o ** 2))
+    else:
+        f_tol = 1e-5 * max(1.0, np.sqrt(np.mean(f_o ** 2))) + 1e-4 * np.abs(f_o)
+    acc = synth.KAPPA / 12.0 * 2.0 * f_tol           # x2: the forces change along the run
+    p_g, v_g = pos.cpu().numpy().astype(np.float64), vel.cpu().numpy().astype(np.float64)
+    dx_bound = 1e-6 * np.abs(p_o) + 1e-5 + (steps * dt) ** 2 * acc
+    dv_bound = 1e-4 * np.abs(v_o) + 1e-7 + steps * dt * acc
+    assert np.all(np.abs(p_g - p_o) <= dx_bound), float((np.abs(p_g - p_o) / dx_bound).max())
+    assert np.all(np.abs(v_g - v_o) <= dv_bound), float((np.abs(v_g - v_o) / dv_bound).max())
+    np.testing.assert_allclose(kin.cpu().numpy(), ekin_o, rtol=1e-3 if precision == 1 else 1e-4)
+    pg32 = pos.cpu().numpy()
+    rp, cl = oracle.neighbors(s, w.model.r_cut, pg32, "cells" if s.periodic else "brute")
+    E_o, F_o, _ = oracle.energy_forces(w.model, w.weights, s, pg32, w.types, rp, cl)
+    check = assert_close16 if precision == 1 else assert_close
+    check(energy.cpu().numpy(), E_o, f"energy at final positions ({integrator})")
+    check(forces.cpu().numpy(), F_o, f"forces at final positions ({integrator})")
+    assert ctx.md_edges() == len(cl)

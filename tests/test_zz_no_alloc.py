@@ -78,3 +78,21 @@ def test_noalloc_reports_capacity_and_rejects_oversize(dev):
     # still correct after the rejected calls
     rp_n, cl_n = _noalloc_list(w, dev, cap=len(cl_a))
     assert np.array_equal(rp_n, rp_a) and np.array_equal(cl_n, cl_a)
+
+
+def test_noalloc_rejects_short_arrays_before_any_launch(dev):
+    # a row_ptr one entry short, or too few positions, is refused by the binding with
+    # INVALID_ARG before the library (and any kernel) sees the pointers
+    from schnet_gnn_molecular_cell_b200 import SNError, Status
+    from schnet_gnn_molecular_cell_b200.binding import build_neighbors_noalloc
+    w = synth.make_workload(1)
+    N = w.system.n_atoms
+    pos = torch.from_numpy(w.pos).to(dev)
+    col = torch.empty(4096, dtype=torch.int32, device=dev)
+    with pytest.raises(SNError) as ei:
+        build_neighbors_noalloc(w.system, w.model.r_cut, pos, torch.empty(N, dtype=torch.int32, device=dev), col)
+    assert ei.value.status == Status.INVALID_ARG
+    with pytest.raises(SNError) as ei:
+        build_neighbors_noalloc(w.system, w.model.r_cut, pos[: N - 1], torch.empty(N + 1, dtype=torch.int32,
+                                                                                  device=dev), col)
+    assert ei.value.status == Status.INVALID_ARG
