@@ -212,6 +212,17 @@ sn_status sn_md_step_host(sn_ctx *ctx, const sn_system *sys, float *pos_host, fl
 sn_status sn_sync(sn_ctx *ctx);
 
 /*
+ * Bound, in GPU clock cycles, of the tensor-core kernels' waits for their own MMAs (default
+ * 2^32, about 2 s; 0 restores it).  These waits depend on no other agent and end in
+ * microseconds; a bound far shorter than an MMA makes them give up: the kernel then latches
+ * SN_ERR_TIMEOUT (returned by the next sn_sync), lets every MMA it issued complete under the
+ * default bound, releases its tensor memory and returns, and later kernels of the call skip
+ * their work.  The context stays usable.  The paper has no counterpart: this exists so that
+ * the time-out path can be exercised.  SN_ERR_INVALID_ARG for a negative bound.
+ */
+sn_status sn_set_wait_limit(sn_ctx *ctx, int64_t cycles);
+
+/*
  * Neighbour list without any device memory allocation.
  *
  * The paper has no counterpart of this entry point; it exists for callers that cannot call

@@ -55,7 +55,7 @@ class TraceEntry(C.Structure):
 EXPORTS = ["sn_create", "sn_destroy", "sn_set_stream", "sn_reserve", "sn_build_neighbors",
            "sn_energy_forces", "sn_md_step", "sn_md_langevin", "sn_md_step_host", "sn_sync", "sn_md_edges",
            "sn_trace_enable", "sn_trace_read", "sn_build_neighbors_noalloc", "sn_last_error",
-           "sn_version"]
+           "sn_version", "sn_set_wait_limit"]
 
 _lib = None
 
@@ -81,6 +81,7 @@ def load():
     L.sn_md_langevin.argtypes = [P, C.POINTER(System), P, P, P, P, f32, f32, i32, f32, f32, C.c_uint64, i64, P, P]
     L.sn_md_langevin.restype = C.c_int
     L.sn_sync.argtypes = [P]
+    L.sn_set_wait_limit.argtypes = [P, i64]
     L.sn_md_edges.argtypes = [P]
     L.sn_md_edges.restype = i64
     L.sn_trace_enable.argtypes = [P, i32]
@@ -93,7 +94,7 @@ def load():
     L.sn_last_error.restype = C.c_char_p
     L.sn_version.restype = C.c_char_p
     for name in ("sn_create", "sn_destroy", "sn_set_stream", "sn_reserve", "sn_build_neighbors",
-                 "sn_energy_forces", "sn_md_step", "sn_md_step_host", "sn_sync"):
+                 "sn_energy_forces", "sn_md_step", "sn_md_step_host", "sn_sync", "sn_set_wait_limit"):
         getattr(L, name).restype = C.c_int
     _lib = L
     return L
@@ -261,6 +262,11 @@ class Context:
 
     def sync(self):
         self._check(self._L.sn_sync(self._h))
+
+    def set_wait_limit(self, cycles: int):
+        """Bound (GPU clock cycles) of the tensor-core kernels' waits for their own MMAs; 0
+        restores the default.  A tiny bound exercises the time-out path (see sn.h)."""
+        self._check(self._L.sn_set_wait_limit(self._h, int(cycles)))
 
     def trace(self, on: bool = True):
         """Enable/disable per-kernel CUDA-event timing (see sn_trace_enable)."""

@@ -43,6 +43,7 @@ struct sn_ctx {
     // device mirrors for sn_md_step_host
     DevBuf hc_pos, hc_vel, hc_forces, hc_types, hc_energy, hc_kin;
     sn::Tracer tracer;
+    long long wait_limit = 1ll << 32;   // bound of the tensor-core kernels' waits for their MMAs
     char last_error[256] = {0};
 };
 
@@ -205,6 +206,7 @@ sn::EfWork ef_work(sn_ctx *ctx)
     w.dst_cap = (int64_t)(ctx->dst.bytes / sizeof(int32_t));
     w.col_cap = 0;
     w.G = edge_grid(ctx);
+    w.wait_limit = ctx->wait_limit;
     return w;
 }
 
@@ -679,6 +681,14 @@ sn_status sn_sync(sn_ctx *ctx)
 {
     if (!ctx) return SN_ERR_INVALID_ARG;
     return drain(ctx);
+}
+
+sn_status sn_set_wait_limit(sn_ctx *ctx, int64_t cycles)
+{
+    if (!ctx) return SN_ERR_INVALID_ARG;
+    if (cycles < 0) return fail(ctx, SN_ERR_INVALID_ARG, "negative wait limit");
+    ctx->wait_limit = cycles == 0 ? (1ll << 32) : (long long)cycles;
+    return SN_OK;
 }
 
 sn_status sn_trace_enable(sn_ctx *ctx, int32_t on)

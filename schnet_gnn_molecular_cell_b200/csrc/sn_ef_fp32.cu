@@ -601,9 +601,10 @@ __global__ void k_partition_rows(const int32_t *__restrict__ row_ptr, int64_t N,
     for (int32_t e = e0 + lane; e < e1; e += 32) dst[e] = (int32_t)i;
 }
 
-EdgeTcArgs tc_args(const EdgeArgs &a, const BlockW &bw, int *d_err)
+EdgeTcArgs tc_args(const EdgeArgs &a, const BlockW &bw, int *d_err, long long wait_limit)
 {
     EdgeTcArgs t{};
+    t.wait_limit = wait_limit;
     t.pos4 = a.pos4;
     t.types = a.types;
     t.row_ptr = a.row_ptr;
@@ -723,6 +724,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
         nt.e2 = m.ro.e2;
         nt.sr1 = m.ro.sr1;
         nt.d_err = d_err;
+        nt.wait_limit = w.wait_limit;
         auto node_args = [&](int t) {
             NodeTcArgs a = nt;
             a.t = t;
@@ -740,7 +742,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
             ea.w = m.blk[t];
             ea.t = t;
             trace_begin(tr, KK_EDGE_FWD, s);
-            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err), KP, split, false, w.G, s))) return e;
+            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err, w.wait_limit), KP, split, false, w.G, s))) return e;
             trace_end(tr, s);
             trace_begin(tr, KK_NODE_FWD, s);
             if ((e = launch_node_tc(node_args(t), split, 0, n_sm, s))) return e;
@@ -756,7 +758,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
             ea.w = m.blk[t];
             ea.t = t;
             trace_begin(tr, KK_EDGE_BWD, s);
-            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err), KP, split, true, w.G, s))) return e;
+            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err, w.wait_limit), KP, split, true, w.G, s))) return e;
             trace_end(tr, s);
         }
         return cudaGetLastError();

@@ -353,6 +353,7 @@ struct Group {
     unsigned char *R;
     uint32_t mbar, tm, lane;
     int i0, i1;
+    long long lim;   // bound of the waits for this group's MMAs
 };
 
 template <int KP, bool SPLIT, int NW>
@@ -369,6 +370,7 @@ __device__ __forceinline__ Group make_group(const EdgeTcArgs &A, unsigned char *
     const int p = blockIdx.x * NW + G.g;
     G.i0 = A.part[p];
     G.i1 = A.part[p + 1];
+    G.lim = A.wait_limit;
     return G;
 }
 
@@ -377,7 +379,7 @@ __device__ __forceinline__ bool wait_weights(const Group &G, unsigned char *sm, 
 {
     using S = TcSmem<KP, SPLIT, NW>;
     uint32_t parity = 0;
-    return wait_mma(G.g, smem_u32(sm + S::WMBAR), parity, d_err);
+    return wait_mma(G.g, smem_u32(sm + S::WMBAR), parity, d_err, G.lim);
 }
 
 // Make this group's shared-memory writes visible to the tensor core, then let thread 0 of the
@@ -393,7 +395,20 @@ __device__ __forceinline__ bool mma_step(const Group &G, uint32_t &phase, int *d
         issue();
         mma_commit(G.mbar);
     }
-    return wait_mma(G.g, G.mbar, phase, d_err);
+    return wait_mma(G.g, G.mbar, phase, d_err, G.lim);
+}
+
+// After a wait gave up: one more commit, whose completion follows that of every MMA the group
+// issued, waited for with the default bound, so that no MMA still writes TMEM when it is freed.
+__device__ __forceinline__ void drain_group(const Group &G, uint32_t &phase, int *d_err)
+{
+    tc_fence_before();
+    wg_sync(G.g);
+    if (G.t == 0) {
+        tc_fence_after();
+        mma_commit(G.mbar);
+    }
+    wait_mma(G.g, G.mbar, phase, d_err, WAIT_BOUND);
 }
 
 // s = ssp(a + b1) from TMEM columns [COL_A, COL_A + TE) into the activation tile
@@ -478,6 +493,8 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
         if (ok) {
             A.H[(int64_t)cur * FF + f] = hacc;
             for (int r = cur + 1; r < G.i1; ++r) A.H[(int64_t)r * FF + f] = 0.0f;   // trailing rows without edges
+        } else {
+            drain_group(G, phase, A.d_err);
         }
     }
     teardown<KP, SPLIT, NW>(sm, tmem0, A.d_err);
@@ -700,6 +717,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
             wg_sync(G.g);
         }
         if (ok && cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
+        if (!ok) drain_group(G, phase, A.d_err);
     }
     teardown<KP, SPLIT, NW>(sm, tmem0, A.d_err);
 }
@@ -762,21 +780,23 @@ struct WsSmem {
 
 // Bounded wait on one barrier phase by every thread of a warp.  A time-out raises the CTA's
 // abort flag, which ends every other wait of the CTA at once; the result is warp-uniform.
-static __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile int *abort, int *d_err)
+static __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, volatile int *abort, int *d_err,
+                                               long long lim)
 {
     const long long t0 = clock64();
     int ok = 1;
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_test_wait(bar, parity)) {
         if (*abort) {
             ok = 0;
             break;
         }
-        if (clock64() - t0 > (1ll << 32)) {
+        if (clock64() - t0 > lim) {
             *abort = 1;
             atomicOr(d_err, ERRBIT_TIMEOUT);
             ok = 0;
             break;
         }
+        if (mbar_try_wait(bar, parity)) break;
     }
     return __all_sync(0xffffffffu, ok) != 0;
 }
@@ -837,7 +857,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
             for (int k = 0; k < nt; ++k) {
                 const int s = k % NSTG, ts = e0 + k * TE, ne = min(TE, e1 - ts);
                 int okw = 1;
-                if (k >= NSTG) okw = ws_wait(bar(WB_FREE, s), ((k / NSTG) - 1) & 1, abort, A.d_err);
+                if (k >= NSTG) okw = ws_wait(bar(WB_FREE, s), ((k / NSTG) - 1) & 1, abort, A.d_err, A.wait_limit);
                 if (!named_sync_and(5, WS_P, okw)) break;   // all P warps go on or stop together
                 const EdgeIdx cidx = nidx;
                 const EdgePos cpos = npos;
@@ -860,7 +880,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
             // M: lane 0 polls the two queues and issues whichever MMA is ready: MMA1 of the next
             // tile whose basis is in (and whose stage E has released), MMA2 of the oldest tile
             // whose activations S has written.  Decisions are broadcast so the warp stays uniform.
-            bool ok = ws_wait(wmbar, 0, abort, A.d_err);
+            bool ok = ws_wait(wmbar, 0, abort, A.d_err, A.wait_limit);
             bool issued = false;
             int k1 = 0, k2 = 0;
             long long last = clock64();
@@ -900,7 +920,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                     last = clock64();
                 } else if (*abort) {
                     ok = false;
-                } else if (clock64() - last > (1ll << 32)) {
+                } else if (clock64() - last > A.wait_limit) {
                     if (lane == 0) {
                         *abort = 1;
                         atomicOr(A.d_err, ERRBIT_TIMEOUT);
@@ -927,7 +947,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
             const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
             for (int k = 0; k < nt; ++k) {
                 const int s = k % NSTG;
-                if (!ws_wait(bar(WB_FULL_A, s), (k / NSTG) & 1, abort, A.d_err)) break;
+                if (!ws_wait(bar(WB_FULL_A, s), (k / NSTG) & 1, abort, A.d_err, A.wait_limit)) break;
                 tc_fence_after();
                 unsigned char *Th = stage(s) + S::T, *Tl = Th + S::TB;
 #pragma unroll 1
@@ -953,9 +973,9 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
             bool ok = true;
             for (int k = 0; k < nt; ++k) {
                 const int s = k % NSTG, ne = min(TE, e1 - (e0 + k * TE));
-                if (!(ok = ws_wait(bar(WB_FULL_W, s), (k / NSTG) & 1, abort, A.d_err))) break;
+                if (!(ok = ws_wait(bar(WB_FULL_W, s), (k / NSTG) & 1, abort, A.d_err, A.wait_limit))) break;
                 // (completed already: P's metadata and the copied source rows are in place)
-                if (!(ok = ws_wait(bar(WB_FULL_B, s), (k / NSTG) & 1, abort, A.d_err))) break;
+                if (!(ok = ws_wait(bar(WB_FULL_B, s), (k / NSTG) & 1, abort, A.d_err, A.wait_limit))) break;
                 tc_fence_after();
                 const float *sXs = reinterpret_cast<const float *>(stage(s) + S::XS) + f;
                 const int *sDst = reinterpret_cast<const int *>(stage(s) + S::DST);

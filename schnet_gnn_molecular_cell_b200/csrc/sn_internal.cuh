@@ -133,6 +133,7 @@ struct EfWork {
     int64_t dst_cap;
     int64_t col_cap;     // entries of this call's col buffer (the list must fit in it)
     int G;
+    long long wait_limit;   // bound (cycles) of the tensor-core kernels' waits for their MMAs
 };
 
 struct Model {
@@ -168,6 +169,7 @@ struct EdgeTcArgs {
     const float *s1, *s2;  // [F] output-channel scales of W1 and W2
     int t;
     int *d_err;
+    long long wait_limit;  // bound (cycles) of the waits for the kernel's own MMAs
 };
 
 cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s);
@@ -192,6 +194,7 @@ struct NodeTcArgs {
     const float *c1, *c2, *e1, *R2, *e2;
     const float *su1, *su2, *sr1;   // output-channel scales of U1, U2 ([F]) and R1 ([128])
     int *d_err;
+    long long wait_limit;           // bound (cycles) of the waits for the kernel's own MMAs
 };
 
 // which: 0 update of block a.t, 1 readout of x^T = X[a.t], 2 backward of block a.t's update

@@ -66,7 +66,8 @@ __device__ __forceinline__ void issue_gemm(unsigned char *W, unsigned char *T, u
 // first GEMM of a CTA waits for them (weights_ready tracks this).
 template <bool SPLIT, bool TRANS>
 __device__ __forceinline__ bool gemm_step(unsigned char *W, unsigned char *T, uint32_t d, uint32_t mbar,
-                                          uint32_t &phase, int *d_err, bool &weights_ready, uint32_t wmbar)
+                                          uint32_t &phase, int *d_err, bool &weights_ready, uint32_t wmbar,
+                                          long long lim)
 {
     if (!weights_ready) {
         if (!wait_copies(wmbar, d_err)) return false;
@@ -80,7 +81,20 @@ __device__ __forceinline__ bool gemm_step(unsigned char *W, unsigned char *T, ui
         issue_gemm<SPLIT, TRANS>(W, T, d);
         mma_commit(mbar);
     }
-    return wait_mma_cta(mbar, phase, d_err);
+    return wait_mma_cta(mbar, phase, d_err, lim);
+}
+
+// After a wait gave up: one more commit, whose completion follows that of every MMA issued,
+// waited for with the default bound before TMEM is freed.
+__device__ __forceinline__ void drain_cta(uint32_t mbar, uint32_t &phase, int *d_err)
+{
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        tc_fence_after();
+        mma_commit(mbar);
+    }
+    wait_mma_cta(mbar, phase, d_err, WAIT_BOUND);
 }
 
 // value(a) for atoms [32g, 32g + 32) of the tile at column f, into the activation tile (zero
@@ -157,10 +171,11 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
     if (!skip) {
         const float c1f = A.c1[f], c2f = A.c2[f], su1f = A.su1[f], su2f = A.su2[f];
         unsigned char *T = sm + S::T;
-        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        bool ok = true;
+        for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
             tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.H[a * FF + f]; });
-            if (!gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar)) break;
+            if (!(ok = gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
@@ -179,7 +194,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
                 const int64_t a = a0 + 32 * c + q;
                 xr[q] = a < A.N ? __ldg(x_row(A, A.t, a) + f) : 0.0f;
             }
-            if (!gemm_step<SPLIT, false>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar)) break;
+            if (!(ok = gemm_step<SPLIT, false>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
@@ -192,6 +207,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
             tc_fence_before();
             __syncthreads();
         }
+        if (!ok) drain_cta(mbar, phase, A.d_err);
     }
     node_teardown(tmem, ready, wmbar, A.d_err);
 }
@@ -217,10 +233,11 @@ __global__ void __launch_bounds__(NT, 1) k_node_readout_tc(NodeTcArgs A)
         const float e1k = f < H ? A.e1[f] : 0.0f, r2k = f < H ? A.R2[f] : 0.0f, e2 = A.e2[0];
         const float sr1k = A.sr1[f], r2s = r2k * sr1k;   // R1's channel scale (1 past H)
         unsigned char *T = sm + S::T;
-        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        bool ok = true;
+        for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
             tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.X[((int64_t)(A.t) * A.N + a) * FF + f]; });
-            if (!gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar)) break;
+            if (!(ok = gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
@@ -232,7 +249,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_readout_tc(NodeTcArgs A)
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
-            if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar)) break;
+            if (!(ok = gemm_step<SPLIT, true>(sm + S::W0, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             if (threadIdx.x < TA) {   // per-atom energy (fixed summation order) and zero forces
                 const int64_t a = a0 + threadIdx.x;
                 if (a < A.N) {
@@ -256,6 +273,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_readout_tc(NodeTcArgs A)
             tc_fence_before();
             __syncthreads();
         }
+        if (!ok) drain_cta(mbar, phase, A.d_err);
     }
     node_teardown(tmem, ready, wmbar, A.d_err);
 }
@@ -279,10 +297,11 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
         unsigned char *T = sm + S::T;
         // the operands of U2^T and U1^T carry the channel scales of U2 and U1
         const float su1f = A.su1[f], su2f = A.su2[f];
-        for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        bool ok = true;
+        for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
             const int64_t a0 = tile * TA;
             tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.Xbar[a * FF + f] * su2f; });
-            if (!gemm_step<SPLIT, true>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar)) break;
+            if (!(ok = gemm_step<SPLIT, true>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
@@ -294,7 +313,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
-            if (!gemm_step<SPLIT, true>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar)) break;
+            if (!(ok = gemm_step<SPLIT, true>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
@@ -307,6 +326,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
             tc_fence_before();
             __syncthreads();
         }
+        if (!ok) drain_cta(mbar, phase, A.d_err);
     }
     node_teardown(tmem, ready, wmbar, A.d_err);
 }

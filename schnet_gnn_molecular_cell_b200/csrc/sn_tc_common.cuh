@@ -136,15 +136,13 @@ static __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, u
 // Bounded wait of the whole CTA for phase 0 of mbar (the weight copies); false on time-out.
 static __device__ __forceinline__ bool wait_copies(uint32_t mbar, int *d_err)
 {
+    int ok = 1;
     const long long t0 = clock64();
-    int ok = 0;
-    for (;;) {
-        if (mbar_try_wait(mbar, 0)) {
-            ok = 1;
+    while (!mbar_try_wait(mbar, 0))
+        if (clock64() - t0 > (1ll << 33)) {
+            ok = 0;
             break;
         }
-        if (clock64() - t0 > (1ll << 33)) break;
-    }
     ok = __syncthreads_and(ok);
     if (!ok && threadIdx.x == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
     return ok != 0;
@@ -296,20 +294,29 @@ static __device__ __forceinline__ int wg_sync_and(int g, int pred)
     return out;
 }
 
-// Bounded wait for the MMAs committed to a warpgroup's mbarrier; every thread of the group
-// calls it at the same point.  On a time-out (never expected: nothing here waits on another
-// agent) the error bit is set and the whole group returns false.
-static __device__ __forceinline__ bool wait_mma(int g, uint32_t mbar, uint32_t &phase, int *d_err)
+// Default bound (GPU clock cycles, about 2 s) of every wait of a kernel for its own MMAs and
+// copies; the context can shorten the MMA waits to exercise the time-out path.
+constexpr long long WAIT_BOUND = 1ll << 32;
+
+// Wait for a barrier phase for at most lim cycles; false on time-out.  The phase is tested
+// before the bound, so that a short bound gives up at once on work still in flight.
+static __device__ __forceinline__ int bounded_phase_wait(uint32_t mbar, uint32_t parity, long long lim)
 {
     const long long t0 = clock64();
-    int ok = 0;
     for (;;) {
-        if (mbar_try_wait(mbar, phase)) {
-            ok = 1;
-            break;
-        }
-        if (clock64() - t0 > (1ll << 33)) break;
+        if (mbar_test_wait(mbar, parity)) return 1;
+        if (clock64() - t0 > lim) return 0;
+        if (mbar_try_wait(mbar, parity)) return 1;
     }
+}
+
+// Bounded wait for the MMAs committed to a warpgroup's mbarrier; every thread of the group
+// calls it at the same point.  On a time-out (never expected with the default bound: nothing
+// here waits on another agent) the error bit is set and the whole group returns false.
+static __device__ __forceinline__ bool wait_mma(int g, uint32_t mbar, uint32_t &phase, int *d_err,
+                                                long long lim = WAIT_BOUND)
+{
+    int ok = bounded_phase_wait(mbar, phase, lim);
     phase ^= 1u;
     ok = wg_sync_and(g, ok);
     if (!ok && (threadIdx.x % WGT) == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
@@ -318,17 +325,10 @@ static __device__ __forceinline__ bool wait_mma(int g, uint32_t mbar, uint32_t &
 }
 
 // The same wait when the whole CTA waits on one mbarrier (every thread calls it).
-static __device__ __forceinline__ bool wait_mma_cta(uint32_t mbar, uint32_t &phase, int *d_err)
+static __device__ __forceinline__ bool wait_mma_cta(uint32_t mbar, uint32_t &phase, int *d_err,
+                                                    long long lim = WAIT_BOUND)
 {
-    const long long t0 = clock64();
-    int ok = 0;
-    for (;;) {
-        if (mbar_try_wait(mbar, phase)) {
-            ok = 1;
-            break;
-        }
-        if (clock64() - t0 > (1ll << 33)) break;
-    }
+    int ok = bounded_phase_wait(mbar, phase, lim);
     phase ^= 1u;
     ok = __syncthreads_and(ok);
     if (!ok && threadIdx.x == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
