@@ -35,7 +35,7 @@ struct sn_ctx {
     int *d_err = nullptr;
     int32_t *h_err = nullptr;          // pinned
     // workspace
-    DevBuf pos4, cnt, cell_of, cell_cnt, cell_start, cell_atoms;
+    DevBuf pos4, cnt, cell_of, cell_cnt, cell_start, cell_atoms, tsum;
     DevBuf x, p, h, hbar, xbar, eps, part, dst;
     DevBuf md_row_ptr, md_col;
     int64_t md_cap = 0;                // entries of md_col
@@ -159,6 +159,7 @@ sn_status ensure_nb(sn_ctx *ctx, const sn_system *s)
     if ((st = grow(ctx, ctx->cell_atoms, sizeof(int32_t) * N))) return st;
     if ((st = grow(ctx, ctx->cell_cnt, sizeof(int32_t) * (ncell + 2)))) return st;
     if ((st = grow(ctx, ctx->cell_start, sizeof(int32_t) * (ncell + 1)))) return st;
+    if ((st = grow(ctx, ctx->tsum, sizeof(int32_t) * ((N > ncell ? N : ncell) / 4096 + 2)))) return st;
     return SN_OK;
 }
 
@@ -187,6 +188,7 @@ sn::NbWork nb_work(sn_ctx *ctx)
     w.cell_cnt = (int32_t *)ctx->cell_cnt.p;
     w.cell_start = (int32_t *)ctx->cell_start.p;
     w.cell_atoms = (int32_t *)ctx->cell_atoms.p;
+    w.tsum = (int32_t *)ctx->tsum.p;
     w.ncell_cap = (int64_t)(ctx->cell_cnt.bytes / sizeof(int32_t)) - 2;
     return w;
 }
@@ -465,7 +467,7 @@ sn_status sn_destroy(sn_ctx *ctx)
 {
     if (!ctx) return SN_ERR_INVALID_ARG;
     cudaStreamSynchronize(ctx->stream);
-    DevBuf *bufs[] = {&ctx->pos4, &ctx->cnt, &ctx->cell_of, &ctx->cell_cnt, &ctx->cell_start, &ctx->cell_atoms,
+    DevBuf *bufs[] = {&ctx->pos4, &ctx->cnt, &ctx->cell_of, &ctx->cell_cnt, &ctx->cell_start, &ctx->cell_atoms, &ctx->tsum,
                       &ctx->x, &ctx->p, &ctx->h, &ctx->hbar, &ctx->xbar, &ctx->eps, &ctx->part, &ctx->dst,
                       &ctx->md_row_ptr, &ctx->md_col, &ctx->hc_pos, &ctx->hc_vel, &ctx->hc_forces,
                       &ctx->hc_types, &ctx->hc_energy, &ctx->hc_kin};

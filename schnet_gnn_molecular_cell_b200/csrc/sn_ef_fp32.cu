@@ -576,6 +576,8 @@ __global__ void k_partition(const int32_t *__restrict__ row_ptr, int64_t N, int 
 __global__ void k_partition_rows(const int32_t *__restrict__ row_ptr, int64_t N, int G, int32_t *__restrict__ part,
                                  unsigned part_blocks, int32_t *__restrict__ dst, int64_t cap, int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     if (blockIdx.x < part_blocks) {
         const int c = blockIdx.x * blockDim.x + threadIdx.x;
         if (c > G) return;
@@ -661,8 +663,9 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
     if (m.precision != SN_PREC_FP32 && N > 0) {
         // one launch: the first blocks partition the rows, the rest index the edges' rows
         const unsigned pb = (unsigned)((parts + 1 + 255) / 256);
-        k_partition_rows<<<pb + (unsigned)((32 * N + 255) / 256), 256, 0, s>>>(
-            row_ptr, N, parts, w.part, pb, w.dst, w.col_cap < w.dst_cap ? w.col_cap : w.dst_cap, d_err);
+        if ((e = launch_pdl(k_partition_rows, dim3(pb + (unsigned)((32 * N + 255) / 256)), dim3(256), 0, s, row_ptr, N,
+                            parts, w.part, pb, w.dst, w.col_cap < w.dst_cap ? w.col_cap : w.dst_cap, d_err)))
+            return e;
     } else {
         k_partition<<<(parts + 1 + 127) / 128, 128, 0, s>>>(row_ptr, N, parts, w.part, w.col_cap, d_err);
     }

@@ -312,8 +312,7 @@ __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm
         for (int g = 0; g < NW; ++g) mbar_init(smem_u32(sm + S::GROUPS + g * S::REGION + S::MBAR), 1);
         mbar_init(wmbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
-        mbar_expect_tx(wmbar, S::NS * (S::W1B + S::W2B));
+        mbar_expect_tx(wmbar, S::NS * (S::W1B + S::W2B));   // constant weights: before the wait
         bulk_g2s(smem_u32(sm + S::W1), A.W1h, S::W1B, wmbar);
         bulk_g2s(smem_u32(sm + S::W2), A.W2h, S::W2B, wmbar);
         if (SPLIT) {
@@ -326,6 +325,10 @@ __device__ __forceinline__ uint32_t setup(const EdgeTcArgs &A, unsigned char *sm
         reinterpret_cast<float *>(sm + S::MUL)[threadIdx.x] = A.basis.mu_lo[threadIdx.x];
     }
     if (warp == 0) tmem_alloc(smem_u32(sm + S::HOLD), 128 * NW);
+    pdl_trigger();
+    pdl_wait();   // from here on: data written by the preceding kernels
+    if (threadIdx.x == 0)
+        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -824,8 +827,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
         mbar_init(drain, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         *abort = 0;
-        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
-        mbar_expect_tx(wmbar, S::NS * (S::W1B + S::W2B));
+        mbar_expect_tx(wmbar, S::NS * (S::W1B + S::W2B));   // constant weights: before the wait
         bulk_g2s(smem_u32(sm + S::W1), A.W1h, S::W1B, wmbar);
         bulk_g2s(smem_u32(sm + S::W2), A.W2h, S::W2B, wmbar);
         if (SPLIT) {
@@ -838,6 +840,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
         reinterpret_cast<float *>(sm + S::MUL)[threadIdx.x] = A.basis.mu_lo[threadIdx.x];
     }
     if (warp == WS_M_WARP) tmem_alloc(smem_u32(sm + S::HOLD), S::TMEM_COLS);
+    pdl_trigger();
+    pdl_wait();   // from here on: data written by the preceding kernels
+    if (threadIdx.x == 0)
+        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1081,18 +1087,18 @@ cudaError_t launch_t(const EdgeTcArgs &a, bool backward, int G, cudaStream_t s)
     cudaError_t e;
     if (backward) {
         if ((e = prepare(k_edge_bwd_tc<KP, SPLIT, NW, CH>, S::BYTES))) return e;
-        k_edge_bwd_tc<KP, SPLIT, NW, CH><<<G, WGT * NW, S::BYTES, s>>>(a);
+        e = launch_pdl(k_edge_bwd_tc<KP, SPLIT, NW, CH>, dim3(G), dim3(WGT * NW), S::BYTES, s, a);
     } else if constexpr (!SPLIT) {
         constexpr int NSTG = 3;
         using WS = WsSmem<KP, false, NSTG>;
         static_assert(WS::BYTES <= 227 * 1024, "shared memory plan exceeds 227 KB");
         if ((e = prepare(k_edge_fwd_ws<KP, false, NSTG, CH>, WS::BYTES))) return e;
-        k_edge_fwd_ws<KP, false, NSTG, CH><<<G, WS_THREADS, WS::BYTES, s>>>(a, NW);
+        e = launch_pdl(k_edge_fwd_ws<KP, false, NSTG, CH>, dim3(G), dim3(WS_THREADS), WS::BYTES, s, a, NW);
     } else {
         if ((e = prepare(k_edge_fwd_tc<KP, SPLIT, NW, CH>, S::BYTES))) return e;
-        k_edge_fwd_tc<KP, SPLIT, NW, CH><<<G, WGT * NW, S::BYTES, s>>>(a);
+        e = launch_pdl(k_edge_fwd_tc<KP, SPLIT, NW, CH>, dim3(G), dim3(WGT * NW), S::BYTES, s, a);
     }
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // The split (fp32-accurate) mode holds two fp16 copies of every operand: two warpgroups fit in

@@ -36,6 +36,35 @@ inline void trace_end(Tracer *t, cudaStream_t s)
     if (t && t->on) t->end(s);
 }
 
+// Programmatic dependent launch.  Kernels of one evaluation or MD step are launched with
+// launch_pdl: a kernel may then start (and do set-up that reads nothing an earlier kernel
+// writes: barrier initialisation, tensor-memory allocation, copies of the constant weights)
+// while its predecessor's last CTAs run.  Every such kernel signals pdl_trigger() as it starts,
+// and calls pdl_wait() on every thread before its first access to data written by an earlier
+// kernel of the stream; pdl_wait returns once the preceding kernels have completed and their
+// writes are visible.  Each kernel waits before it ends, so completion stays transitive along
+// the chain.  (A dependent grid launches only once every CTA of its predecessor has started.)
+#ifdef __CUDACC__
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+#endif
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Conditions latched on the device in ctx->d_err (bitwise OR).  Kernels that run after a
 // latched condition return without touching memory.
 enum : int {
@@ -109,6 +138,7 @@ struct NbWork {
     int32_t *cell_cnt; // [ncell + 2]: counts / cursors, then (last entry) the stencil flag
     int32_t *cell_start; // [ncell + 1]
     int32_t *cell_atoms; // [N]
+    int32_t *tsum;       // [max(N, ncell) / 4096 + 2]: per-tile sums of the multi-CTA scans
     int64_t ncell_cap;
 };
 

@@ -30,6 +30,8 @@ __device__ __forceinline__ void store_pos4(float4 *pos4, int64_t i, const float 
 __global__ void k_kick_drift(float *__restrict__ pos, float *__restrict__ vel, const float *__restrict__ forces,
                              int64_t N, float c, float dt, float4 *__restrict__ pos4, int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     if (skip_all(d_err)) return;
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= N) return;
@@ -48,6 +50,8 @@ __global__ void k_kick_drift(float *__restrict__ pos, float *__restrict__ vel, c
 __global__ void k_kick(float *__restrict__ vel, const float *__restrict__ forces, int64_t n3, float c,
                        const int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     if (skip_all(d_err)) return;
     int64_t q = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (q >= n3) return;
@@ -60,6 +64,8 @@ __global__ void __launch_bounds__(RB) k_replica_sums(const float *__restrict__ e
                                                      float *__restrict__ kinetic, const int *__restrict__ d_err)
 {
     __shared__ float se[RB], sk[RB];
+    pdl_trigger();
+    pdl_wait();
     if (skip_all(d_err)) return;
     const int r = blockIdx.x;
     const int64_t base = (int64_t)r * n_per;
@@ -130,6 +136,8 @@ __global__ void k_langevin_baoa(float *__restrict__ pos, float *__restrict__ vel
                                 int64_t N, float c, float dt, float a, float b, uint64_t seed, int64_t step,
                                 float4 *__restrict__ pos4, int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     if (skip_all(d_err)) return;
     const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= N) return;
@@ -158,9 +166,10 @@ cudaError_t launch_langevin_baoa(float *pos, float *vel, const float *forces, in
 {
     if (N == 0) return cudaSuccess;
     trace_begin(tr, KK_KICK_DRIFT, s);
-    k_langevin_baoa<<<blocks_for(N, 128), 128, 0, s>>>(pos, vel, forces, N, c, dt, a, b, seed, step, pos4, d_err);
+    cudaError_t e = launch_pdl(k_langevin_baoa, dim3(blocks_for(N, 128)), dim3(128), 0, s, pos, vel, forces, N, c, dt, a,
+                               b, seed, step, pos4, d_err);
     trace_end(tr, s);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64_t N, float c, float dt,
@@ -168,9 +177,10 @@ cudaError_t launch_kick_drift(float *pos, float *vel, const float *forces, int64
 {
     if (N == 0) return cudaSuccess;
     trace_begin(tr, KK_KICK_DRIFT, s);
-    k_kick_drift<<<blocks_for(N, 256), 256, 0, s>>>(pos, vel, forces, N, c, dt, pos4, d_err);
+    cudaError_t e = launch_pdl(k_kick_drift, dim3(blocks_for(N, 256)), dim3(256), 0, s, pos, vel, forces, N, c, dt, pos4,
+                               d_err);
     trace_end(tr, s);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_kick(float *vel, const float *forces, int64_t n3, float c, int *d_err, cudaStream_t s,
@@ -178,9 +188,9 @@ cudaError_t launch_kick(float *vel, const float *forces, int64_t n3, float c, in
 {
     if (n3 == 0) return cudaSuccess;
     trace_begin(tr, KK_KICK, s);
-    k_kick<<<blocks_for(n3, 256), 256, 0, s>>>(vel, forces, n3, c, d_err);
+    cudaError_t e = launch_pdl(k_kick, dim3(blocks_for(n3, 256)), dim3(256), 0, s, vel, forces, n3, c, d_err);
     trace_end(tr, s);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_replica_sums(const float *eps, const float *vel, int n_per, int n_rep, float half_m_over_kappa,
@@ -188,9 +198,10 @@ cudaError_t launch_replica_sums(const float *eps, const float *vel, int n_per, i
 {
     if (n_rep == 0) return cudaSuccess;
     trace_begin(tr, KK_SUMS, s);
-    k_replica_sums<<<n_rep, RB, 0, s>>>(eps, vel, n_per, half_m_over_kappa, energy, kinetic, d_err);
+    cudaError_t e = launch_pdl(k_replica_sums, dim3(n_rep), dim3(RB), 0, s, eps, vel, n_per, half_m_over_kappa, energy,
+                               kinetic, d_err);
     trace_end(tr, s);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace sn

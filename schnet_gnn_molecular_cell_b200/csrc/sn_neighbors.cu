@@ -54,6 +54,8 @@ __device__ __forceinline__ float pair_r2(float4 pi, float4 pj, const Geometry &g
 __global__ void k_prep_positions(const float *__restrict__ pos, float4 *__restrict__ pos4, int64_t N,
                                  int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= N) return;
     float x = pos[3 * i], y = pos[3 * i + 1], z = pos[3 * i + 2];
@@ -75,6 +77,8 @@ __global__ void __launch_bounds__(256) k_pairs(const float4 *__restrict__ pos4, 
                                                int32_t *__restrict__ col, int64_t cap, int64_t N,
                                                int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (i >= N) return;
@@ -130,6 +134,8 @@ __global__ void k_cell_assign(const float4 *__restrict__ pos4, int64_t N, Geomet
                               int32_t *__restrict__ cell_of, int32_t *__restrict__ cell_cnt,
                               const int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= N || (*((volatile const int *)d_err) & ERRBIT_NONFINITE)) return;
     float4 p = pos4[i];
@@ -145,6 +151,8 @@ __global__ void k_cell_assign(const float4 *__restrict__ pos4, int64_t N, Geomet
 __global__ void k_cell_scatter(int64_t N, const int32_t *__restrict__ cell_of, int32_t *__restrict__ cursor,
                                int32_t *__restrict__ cell_atoms, const int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i >= N || (*((volatile const int *)d_err) & ERRBIT_NONFINITE)) return;
     int32_t slot = atomicAdd(&cursor[cell_of[i]], 1);
@@ -159,6 +167,8 @@ __global__ void __launch_bounds__(BT) k_cell_pairs(const float4 *__restrict__ po
                                                    int32_t *__restrict__ cnt, const int32_t *__restrict__ row_ptr,
                                                    int32_t *__restrict__ col, int64_t cap, int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     if (*((volatile int *)d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) return;
     if (FILL && (int64_t)row_ptr[N] > cap) {
         if (threadIdx.x == 0 && blockIdx.x == 0) atomicOr(d_err, ERRBIT_CAPACITY);
@@ -230,66 +240,11 @@ __global__ void __launch_bounds__(BT) k_cell_pairs(const float4 *__restrict__ po
 }
 
 // -------------------------------------------------------------------- exclusive scan
-// One CTA of 1024 threads: out[0] = 0, out[k+1] = sum_{q<=k} in[q] for k < n.  Sums above
-// INT32_MAX latch ERRBIT_CAPACITY (a list that large cannot be indexed by int32).
-// out[0] = 0, out[q + 1] = in[0] + .. + in[q] (exclusive scan into n + 1 entries), by one
-// CTA of 1024 threads over tiles of 4096 entries (4 consecutive per thread), carrying the
-// running total from tile to tile; sums beyond int32 latch the capacity condition.
-__global__ void __launch_bounds__(1024) k_scan(const int32_t *__restrict__ in, int32_t *__restrict__ out, int64_t n,
-                                               int *__restrict__ d_err)
-{
-    __shared__ long long warp_sums[32];
-    const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
-    if (t == 0) out[0] = 0;
-    long long carry = 0;
-    bool over = false;
-    int nv[4];   // the next tile's entries, loaded while the current one is scanned
-#pragma unroll
-    for (int k = 0; k < 4; ++k) nv[k] = 4 * t + k < n ? in[4 * t + k] : 0;
-    for (int64_t tile = 0; tile < n; tile += 4096) {
-        const int64_t q0 = tile + 4 * t;
-        int v[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            v[k] = nv[k];
-            nv[k] = q0 + 4096 + k < n ? in[q0 + 4096 + k] : 0;
-        }
-        const long long s = (long long)v[0] + v[1] + v[2] + v[3];
-        long long x = s;   // inclusive scan of the thread sums within the warp
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const long long y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane == 31) warp_sums[wid] = x;
-        __syncthreads();
-        if (wid == 0) {
-            long long ws = warp_sums[lane];
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const long long y = __shfl_up_sync(0xffffffffu, ws, o);
-                if (lane >= o) ws += y;
-            }
-            warp_sums[lane] = ws;
-        }
-        __syncthreads();
-        long long run = carry + x - s + (wid > 0 ? warp_sums[wid - 1] : 0);
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-            if (q0 + k < n) {
-                run += v[k];
-                over |= run > 0x7fffffffLL;
-                out[q0 + k + 1] = (int32_t)(run > 0x7fffffffLL ? 0x7fffffff : run);
-            }
-        carry += warp_sums[31];
-        __syncthreads();   // warp_sums is rewritten by the next tile
-    }
-    if (over) atomicOr(d_err, ERRBIT_CAPACITY);
-}
-
-// The same exclusive scan over many CTAs, in two launches: k_scan_tiles scans each 4096-entry
-// tile in its own CTA (tile-local sums into out, tile totals into tsum); k_scan_add adds the
-// totals of the earlier tiles.  Used where a scratch array of ceil(n / 4096) entries is free.
+// out[0] = 0, out[q + 1] = in[0] + .. + in[q] (exclusive scan into n + 1 entries) over many
+// CTAs, in two launches: k_scan_tiles scans each 4096-entry tile in its own CTA (4 consecutive
+// entries per thread; tile-local sums into out, tile totals into tsum); k_scan_add adds the
+// totals of the earlier tiles.  Sums beyond int32 latch the capacity condition (a list that
+// large cannot be indexed by int32).
 __device__ __forceinline__ long long block_scan_1024(long long s, long long &total, long long *warp_sums)
 {
     const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
@@ -318,6 +273,8 @@ __device__ __forceinline__ long long block_scan_1024(long long s, long long &tot
 __global__ void __launch_bounds__(1024) k_scan_tiles(const int32_t *__restrict__ in, int32_t *__restrict__ out,
                                                      int64_t n, int32_t *__restrict__ tsum)
 {
+    pdl_trigger();
+    pdl_wait();
     __shared__ long long warp_sums[32];
     const int t = threadIdx.x;
     const int64_t q0 = (int64_t)blockIdx.x * 4096 + 4 * t;
@@ -341,6 +298,8 @@ __global__ void __launch_bounds__(1024) k_scan_tiles(const int32_t *__restrict__
 __global__ void __launch_bounds__(1024) k_scan_add(int32_t *__restrict__ out, int64_t n,
                                                    const int32_t *__restrict__ tsum, int *__restrict__ d_err)
 {
+    pdl_trigger();
+    pdl_wait();
     __shared__ long long part[32];
     const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
     long long off = 0;
@@ -367,8 +326,20 @@ __global__ void __launch_bounds__(1024) k_scan_add(int32_t *__restrict__ out, in
 
 __global__ void k_copy_i32(const int32_t *__restrict__ a, int32_t *__restrict__ b, int64_t n)
 {
+    pdl_trigger();
+    pdl_wait();
     int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
     if (i < n) b[i] = a[i];
+}
+
+// out[0] = 0, out[q + 1] = in[0] + .. + in[q] for q < n, over ceil(n / 4096) CTAs in two launches
+cudaError_t scan(const int32_t *in, int32_t *out, int64_t n, int32_t *tsum, int *d_err, cudaStream_t s)
+{
+    const unsigned tiles = (unsigned)((n + 4095) / 4096);
+    if (tiles == 0) return cudaMemsetAsync(out, 0, sizeof(int32_t), s);
+    cudaError_t e = launch_pdl(k_scan_tiles, dim3(tiles), dim3(1024), 0, s, in, out, n, tsum);
+    if (e == cudaSuccess) e = launch_pdl(k_scan_add, dim3(tiles), dim3(1024), 0, s, out, n, (const int32_t *)tsum, d_err);
+    return e;
 }
 
 bool use_cells(const sn_system &sys, float r_cut, int nc[3])
@@ -396,9 +367,9 @@ cudaError_t launch_prep_positions(const float *pos, float4 *pos4, int64_t N, int
 {
     if (N == 0) return cudaSuccess;
     trace_begin(tr, KK_PREP, s);
-    k_prep_positions<<<blocks_for(N, 256), 256, 0, s>>>(pos, pos4, N, d_err);
+    cudaError_t e = launch_pdl(k_prep_positions, dim3(blocks_for(N, 256)), dim3(256), 0, s, pos, pos4, N, d_err);
     trace_end(tr, s);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *pos4, NbWork &w,
@@ -441,30 +412,31 @@ cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *po
         cg.flag = w.cell_cnt + ncell + 1;
         if ((e = cudaMemsetAsync(w.cell_cnt, 0, sizeof(int32_t) * (ncell + 2), s))) return e;
         trace_begin(tr, KK_CELLS, s);
-        k_cell_assign<<<blocks_for(N, 256), 256, 0, s>>>(pos4, N, g, cg, w.cell_of, w.cell_cnt, d_err);
-        k_scan<<<1, 1024, 0, s>>>(w.cell_cnt, w.cell_start, ncell, d_err);
+        if ((e = launch_pdl(k_cell_assign, dim3(blocks_for(N, 256)), dim3(256), 0, s, pos4, N, g, cg, w.cell_of,
+                            w.cell_cnt, d_err)))
+            return e;
+        if ((e = scan(w.cell_cnt, w.cell_start, ncell, w.tsum, d_err, s))) return e;
         // cursor = cell_start (reuse cell_cnt as the cursor array)
-        k_copy_i32<<<blocks_for(ncell, 256), 256, 0, s>>>(w.cell_start, w.cell_cnt, ncell);
-        k_cell_scatter<<<blocks_for(N, 256), 256, 0, s>>>(N, w.cell_of, w.cell_cnt, w.cell_atoms, d_err);
+        if ((e = launch_pdl(k_copy_i32, dim3(blocks_for(ncell, 256)), dim3(256), 0, s, w.cell_start, w.cell_cnt, ncell)))
+            return e;
+        if ((e = launch_pdl(k_cell_scatter, dim3(blocks_for(N, 256)), dim3(256), 0, s, N, w.cell_of, w.cell_cnt,
+                            w.cell_atoms, d_err)))
+            return e;
         trace_end(tr, s);
         trace_begin(tr, KK_NB_COUNT, s);
-        k_cell_pairs<false><<<blocks_for(N, BT), BT, 0, s>>>(pos4, N, g, cg, rc2, w.cell_of, w.cell_start,
-                                                             w.cell_atoms, w.cnt, row_ptr, col, cap, d_err);
+        if ((e = launch_pdl(k_cell_pairs<false>, dim3(blocks_for(N, BT)), dim3(BT), 0, s, pos4, N, g, cg, rc2,
+                            w.cell_of, w.cell_start, w.cell_atoms, w.cnt, row_ptr, col, cap, d_err)))
+            return e;
         trace_end(tr, s);
     } else {
         trace_begin(tr, KK_NB_COUNT, s);
-        k_pairs<false><<<blocks_for(32 * N, 256), 256, 0, s>>>(pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col,
-                                                                cap, N, d_err);
+        if ((e = launch_pdl(k_pairs<false>, dim3(blocks_for(32 * N, 256)), dim3(256), 0, s, pos4, sys.n_per_replica, g,
+                            rc2, w.cnt, row_ptr, col, cap, N, d_err)))
+            return e;
         trace_end(tr, s);
     }
     trace_begin(tr, KK_SCAN, s);
-    if (!cells) {   // row offsets over many CTAs (cell_of is free scratch on this path)
-        const unsigned tiles = (unsigned)((N + 4095) / 4096);
-        k_scan_tiles<<<tiles, 1024, 0, s>>>(w.cnt, row_ptr, N, w.cell_of);
-        k_scan_add<<<tiles, 1024, 0, s>>>(row_ptr, N, w.cell_of, d_err);
-    } else {
-        k_scan<<<1, 1024, 0, s>>>(w.cnt, row_ptr, N, d_err);
-    }
+    if ((e = scan(w.cnt, row_ptr, N, w.tsum, d_err, s))) return e;
     trace_end(tr, s);
     if ((e = cudaGetLastError())) return e;
     if (n_edges_host) {
@@ -476,11 +448,13 @@ cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *po
     }
     trace_begin(tr, KK_NB_FILL, s);
     if (cells) {
-        k_cell_pairs<true><<<blocks_for(N, BT), BT, 0, s>>>(pos4, N, g, cg, rc2, w.cell_of, w.cell_start,
-                                                            w.cell_atoms, w.cnt, row_ptr, col, cap, d_err);
+        if ((e = launch_pdl(k_cell_pairs<true>, dim3(blocks_for(N, BT)), dim3(BT), 0, s, pos4, N, g, cg, rc2, w.cell_of,
+                            w.cell_start, w.cell_atoms, w.cnt, row_ptr, col, cap, d_err)))
+            return e;
     } else {
-        k_pairs<true><<<blocks_for(32 * N, 256), 256, 0, s>>>(pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col,
-                                                               cap, N, d_err);
+        if ((e = launch_pdl(k_pairs<true>, dim3(blocks_for(32 * N, 256)), dim3(256), 0, s, pos4, sys.n_per_replica, g,
+                            rc2, w.cnt, row_ptr, col, cap, N, d_err)))
+            return e;
     }
     trace_end(tr, s);
     return cudaGetLastError();

@@ -27,7 +27,9 @@ constexpr size_t kOffCellOf = align256(kOffCnt + sizeof(int32_t) * (kMaxAtoms + 
 constexpr size_t kOffCellAtoms = align256(kOffCellOf + sizeof(int32_t) * kMaxAtoms);
 constexpr size_t kOffCellCnt = align256(kOffCellAtoms + sizeof(int32_t) * kMaxAtoms);   // [kMaxCells + 2]
 constexpr size_t kOffCellStart = align256(kOffCellCnt + sizeof(int32_t) * (kMaxCells + 2));
-constexpr size_t kOffErr = align256(kOffCellStart + sizeof(int32_t) * (kMaxCells + 1)); // int32 error bits
+constexpr size_t kOffTsum = align256(kOffCellStart + sizeof(int32_t) * (kMaxCells + 1));  // scan tile sums
+constexpr int64_t kTsum = (kMaxAtoms > kMaxCells ? kMaxAtoms : kMaxCells) / 4096 + 2;
+constexpr size_t kOffErr = align256(kOffTsum + sizeof(int32_t) * kTsum);                // int32 error bits
 constexpr size_t kScratchBytes = align256(kOffErr + sizeof(int32_t));
 
 static __device__ __align__(256) unsigned char g_nb_scratch[kScratchBytes];
@@ -77,6 +79,7 @@ extern "C" sn_status sn_build_neighbors_noalloc(const sn_system *sys, float r_cu
     w.cell_atoms = reinterpret_cast<int32_t *>(base + kOffCellAtoms);
     w.cell_cnt = reinterpret_cast<int32_t *>(base + kOffCellCnt);
     w.cell_start = reinterpret_cast<int32_t *>(base + kOffCellStart);
+    w.tsum = reinterpret_cast<int32_t *>(base + kOffTsum);
     w.ncell_cap = kMaxCells;
     int *d_err = reinterpret_cast<int *>(base + kOffErr);
 

@@ -128,8 +128,7 @@ __device__ __forceinline__ uint32_t node_setup(const NodeTcArgs &A, unsigned cha
         mbar_init(smem_u32(sm + S::MBAR), 1);
         mbar_init(wmbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
-        mbar_expect_tx(wmbar, S::NS * S::WB * (w1h ? 2 : 1));
+        mbar_expect_tx(wmbar, S::NS * S::WB * (w1h ? 2 : 1));   // constant weights: before the wait
         bulk_g2s(smem_u32(sm + S::W0), w0h, S::WB, wmbar);
         if (SPLIT) bulk_g2s(smem_u32(sm + S::W0 + S::WB), w0l, S::WB, wmbar);
         if (w1h) {
@@ -138,6 +137,10 @@ __device__ __forceinline__ uint32_t node_setup(const NodeTcArgs &A, unsigned cha
         }
     }
     if ((threadIdx.x >> 5) == 0) tmem_alloc(smem_u32(sm + S::HOLD), 256);
+    pdl_trigger();
+    pdl_wait();   // from here on: data written by the preceding kernels
+    if (threadIdx.x == 0)
+        skip = (*((volatile const int *)A.d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY | ERRBIT_TIMEOUT)) != 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -336,8 +339,7 @@ cudaError_t launch_k(Kern k, uint32_t bytes, int grid, const NodeTcArgs &a, cuda
 {
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
-    k<<<grid, NT, bytes, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(k, dim3(grid), dim3(NT), bytes, s, a);
 }
 
 }  // namespace
