@@ -228,7 +228,7 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
     unsigned char *Bh = R + S::B;
     unsigned char *Bl = Bh + S::BB;
     const uint32_t row = (uint32_t)((n & 7) * 16 + (n >> 3) * S::SW1);
-#pragma unroll
+#pragma unroll 1
     for (int qq = 0; qq < KP / (8 * PARTS); ++qq) {
         const int q = half * (KP / (8 * PARTS)) + qq;
         float v[8];
@@ -449,25 +449,32 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
         float hacc = 0.0f;
         // h_i += x_src (.) (w + b2) over one chunk of CH edges, running sums per destination
         // row; a row is written when the next one starts (rows in between have no edges)
-        auto chunk = [&](int c, int ne, auto full) {
-            constexpr bool FULL = decltype(full)::value;
+        // (one pass per row segment of the chunk, the row change in the code once; padding
+        // edges gather row 0 and are not summed)
+        const uint32_t *sMask = reinterpret_cast<const uint32_t *>(G.R + S::MASK);
+        auto chunk = [&](int c, int ne, uint64_t starts) {
             float v[CH], xs[CH];
             tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, v);
 #pragma unroll
             for (int q = 0; q < CH; ++q) xs[q] = __ldg(xbase + sXo[CH * c + q]);
+            const uint32_t m = (uint32_t)(starts >> (CH * c)) & (CH >= 32 ? 0xffffffffu : (1u << (CH & 31)) - 1u);
+            const int qend = min(CH, ne - CH * c);
+            uint32_t rem = m;
+            int q0 = 0;
+#pragma unroll 1
+            for (;;) {
+                const int q1 = rem ? __ffs(rem) - 1 : qend;
 #pragma unroll
-            for (int q = 0; q < CH; ++q) {
-                const int n = CH * c + q;
-                if (FULL || n < ne) {
-                    const int i = sDst[n];
-                    if (i != cur) {
-                        A.H[(int64_t)cur * FF + f] = hacc;
-                        for (int r = cur + 1; r < i; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
-                        hacc = 0.0f;
-                        cur = i;
-                    }
-                    hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
-                }
+                for (int q = 0; q < CH; ++q)
+                    if (q >= q0 && q < q1) hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
+                if (!rem) break;
+                const int i = sDst[CH * c + q1];
+                A.H[(int64_t)cur * FF + f] = hacc;
+                for (int r = cur + 1; r < i; ++r) A.H[(int64_t)r * FF + f] = 0.0f;
+                hacc = 0.0f;
+                cur = i;
+                rem &= rem - 1u;
+                q0 = q1;
             }
         };
         bool ok = true;
@@ -485,11 +492,10 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_fwd_tc(EdgeTcArgs A)
             if (more) npos = load_pos(A, nidx);
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, false>(sm, G.R, G.tm + COL_W); })))
                 break;
+            const uint64_t starts = (uint64_t)sMask[0] | ((uint64_t)sMask[1] << 32);
 #pragma unroll 1
-            for (int c = 0; c < TE / CH; ++c) {
-                if (CH * c + CH <= ne) chunk(c, ne, std::true_type{});
-                else if (CH * c < ne) chunk(c, ne, std::false_type{});
-            }
+            for (int c = 0; c < TE / CH; ++c)
+                if (CH * c < ne) chunk(c, ne, starts);
             tc_fence_before();
             wg_sync(G.g);
         }
@@ -537,19 +543,26 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
         // scale s2 (wbar s2 = x_j (hbar_i s2) + (x_i s2) hbar_j).
         int cur = -1, nrow = -1;
         float xbacc = 0.0f, xbold = 0.0f, xi_c = 0.0f, hi_c = 0.0f, nxb = 0.0f, nxi = 0.0f, nhi = 0.0f;
-        auto next_row = [&](int i) {
-            if (cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
-            xbacc = 0.0f;
-            cur = i;
+        // the values of row i (read ahead when it is cur + 1): xbar^{t+1}_i, x_i s2, hbar_i s2
+        auto row_vals = [&](int i, float &xb, float &xi, float &hi) {
             if (i == nrow) {
-                xbold = nxb;
-                xi_c = nxi * s2f;
-                hi_c = nhi * s2f;
+                xb = nxb;
+                xi = nxi * s2f;
+                hi = nhi * s2f;
             } else {
-                xbold = A.Xbar[(int64_t)i * FF + f];
-                xi_c = __ldg(x_row(A, xbase, i)) * s2f;
-                hi_c = __ldg(hbase + (int64_t)i * FF) * s2f;
+                xb = A.Xbar[(int64_t)i * FF + f];
+                xi = __ldg(x_row(A, xbase, i)) * s2f;
+                hi = __ldg(hbase + (int64_t)i * FF) * s2f;
             }
+        };
+        // row i starts with the values (xb, xi, hi); the previous row's xbar is written
+        auto open_row = [&](int i, float xb, float xi, float hi, float sum) {
+            if (cur >= 0) A.Xbar[(int64_t)cur * FF + f] = xbold + xbacc;
+            xbacc = sum;
+            cur = i;
+            xbold = xb;
+            xi_c = xi;
+            hi_c = hi;
             nrow = i + 1 < A.N ? i + 1 : -1;
             if (nrow >= 0) {   // discarded unless row i + 1 is this group's next row; the loads
                                // stay here (ld_keep) and are scaled when the row starts
@@ -558,12 +571,17 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 nhi = ldnc_keep(hbase + (int64_t)nrow * FF);
             }
         };
+        auto next_row = [&](int i) {
+            float xb, xi, hi;
+            row_vals(i, xb, xi, hi);
+            open_row(i, xb, xi, hi, 0.0f);
+        };
         // xbar_i += hbar_j (.) (w + b2) and the tile of wbar = x_j (.) hbar_i + x_i (.) hbar_j over
         // one chunk of CH edges (zero for padding edges)
         // A row changes exactly at the edges that start their row (the tile's row-start mask), so
         // chunks without a start skip the row bookkeeping.
-        auto chunk = [&](int c, int ne, uint64_t starts, auto full) {
-            constexpr bool FULL = decltype(full)::value;
+        // (padding edges gather row 0, whose values are then discarded)
+        auto chunk = [&](int c, int ne, uint64_t starts) {
             float w[CH], hb[CH], xj[CH];
             tmem_ld<CH>(G.tm + G.lane + COL_W + CH * c, w);
 #pragma unroll
@@ -573,24 +591,53 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 hb[q] = __ldg(hbase + o.y);
             }
             const uint32_t m = (uint32_t)(starts >> (CH * c)) & (CH >= 32 ? 0xffffffffu : (1u << (CH & 31)) - 1u);
-            if (FULL && m == 0) {
+            const int qend = min(CH, ne - CH * c);   // valid edges of the chunk (>= 1)
+            if (qend == CH && m == 0) {
 #pragma unroll
                 for (int q = 0; q < CH; ++q) {
                     xbacc = fmaf(hb[q], fmaf(w[q], s2f, b2f), xbacc);
                     xj[q] = xj[q] * hi_c + xi_c * hb[q];
                 }
-            } else {
+            } else if (qend == CH && (m & (m - 1u)) == 0) {
+                // one row starts at edge p: edges before it finish row cur, edges from it use the
+                // new row's values (two running sums, one pass)
+                const int p = __ffs(m) - 1, r = sDst[CH * c + p];
+                float xb, xi, hi;
+                row_vals(r, xb, xi, hi);
+                float a0 = xbacc, b0 = 0.0f;
 #pragma unroll
                 for (int q = 0; q < CH; ++q) {
-                    const int n = CH * c + q;
-                    if (FULL || n < ne) {
-                        if ((m >> q) & 1u) next_row(sDst[n]);
-                        xbacc = fmaf(hb[q], fmaf(w[q], s2f, b2f), xbacc);
-                        xj[q] = xj[q] * hi_c + xi_c * hb[q];
-                    } else {
-                        xj[q] = 0.0f;
-                    }
+                    const bool before = q < p;
+                    const float t0 = fmaf(hb[q], fmaf(w[q], s2f, b2f), before ? a0 : b0);
+                    a0 = before ? t0 : a0;
+                    b0 = before ? b0 : t0;
+                    xj[q] = xj[q] * (before ? hi_c : hi) + (before ? xi_c : xi) * hb[q];
                 }
+                xbacc = a0;
+                open_row(r, xb, xi, hi, b0);
+            } else {
+                // row starts (or the ragged end of the list) in the chunk: one pass per row
+                // segment [q0, q1) over the whole chunk under a predicate, so that the row change
+                // is in the code once (the mask holds valid edges only)
+                uint32_t rem = m;
+                int q0 = 0;
+#pragma unroll 1
+                for (;;) {
+                    const int q1 = rem ? __ffs(rem) - 1 : qend;
+#pragma unroll
+                    for (int q = 0; q < CH; ++q)
+                        if (q >= q0 && q < q1) {
+                            xbacc = fmaf(hb[q], fmaf(w[q], s2f, b2f), xbacc);
+                            xj[q] = xj[q] * hi_c + xi_c * hb[q];
+                        }
+                    if (!rem) break;
+                    next_row(sDst[CH * c + q1]);
+                    rem &= rem - 1u;
+                    q0 = q1;
+                }
+#pragma unroll
+                for (int q = 0; q < CH; ++q)
+                    if (q >= qend) xj[q] = 0.0f;
             }
             store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, xj);
         };
@@ -611,8 +658,14 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
             const uint64_t starts = (uint64_t)sMask[0] | ((uint64_t)sMask[1] << 32);
 #pragma unroll 1
             for (int c = 0; c < TE / CH; ++c) {
-                if (CH * c + CH <= ne) chunk(c, ne, starts, std::true_type{});
-                else chunk(c, ne, starts, std::false_type{});
+                if (CH * c < ne) {
+                    chunk(c, ne, starts);
+                } else {   // no edge of the chunk: zero wbar columns
+                    float z[CH];
+#pragma unroll
+                    for (int q = 0; q < CH; ++q) z[q] = 0.0f;
+                    store_tile_col<SPLIT, CH>(Th, Tl, f, CH * c, z);
+                }
             }
             if (!(ok = mma_step(G, phase, A.d_err, [&] { issue_mma_w2<S, SPLIT, true>(sm, G.R, G.tm + COL_W); })))
                 break;
@@ -650,7 +703,7 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
                 const float *mh = reinterpret_cast<const float *>(sm + S::MUH) + par;
                 const float *ml = reinterpret_cast<const float *>(sm + S::MUL) + par;
                 float gsum = 0.0f;
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < KP / 32; ++c) {
                     float gg[16];
                     tmem_ld16x64b_x16(G.tm + G.lane + COL_A + 32 * c, gg);
@@ -987,24 +1040,25 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                 const int *sDst = reinterpret_cast<const int *>(stage(s) + S::DST);
                 const uint32_t *sMask = reinterpret_cast<const uint32_t *>(stage(s) + S::MASK);
                 const uint64_t starts = (uint64_t)sMask[0] | ((uint64_t)sMask[1] << 32);
-                // A full tile with no row without edges inside takes the branch-free path: the
-                // finished row is stored under a predicate at each row start.
-                const bool fast = ne == TE && (sMask[2] | sMask[3]) == 0;
-                auto chunk = [&](int c, auto full) {
-                    constexpr bool FAST = decltype(full)::value;
+                // h of the rows started in the chunk: one pass per row segment [q0, q1) over the
+                // whole chunk under a predicate, so that the row change is in the code once; a
+                // finished row is written when the next starts, rows in between (without edges)
+                // receive zero
+                auto chunk = [&](int c) {
                     float v[CH], xs[CH];
                     tmem_ld<CH>(tmem + lanes + 64 * s + CH * c, v);
 #pragma unroll
                     for (int q = 0; q < CH; ++q) xs[q] = sXs[(CH * c + q) * FF];
                     const uint32_t m = (uint32_t)(starts >> (CH * c)) & (CH >= 32 ? 0xffffffffu : (1u << (CH & 31)) - 1u);
-                    if (FAST && m == 0) {   // the chunk continues the current row
+                    const int qend = min(CH, ne - CH * c);   // valid edges of the chunk (>= 1)
+                    if (qend == CH && m == 0) {   // the chunk continues the current row
 #pragma unroll
                         for (int q = 0; q < CH; ++q) hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
                         return;
                     }
-                    if (FAST && (m & (m - 1u)) == 0) {
+                    if (qend == CH && (m & (m - 1u)) == 0) {
                         // one row starts at edge p of the chunk: edges before it finish row cur,
-                        // edges from it open the next row (two running sums, one store)
+                        // edges from it open the next row (two running sums, one pass)
                         const int p = __ffs(m) - 1;
                         float a0 = hacc, b0 = 0.0f;
 #pragma unroll
@@ -1014,42 +1068,34 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                             a0 = before ? t0 : a0;
                             b0 = before ? b0 : t0;
                         }
+                        const int r = sDst[CH * c + p];
                         store_if(A.H + (int64_t)cur * FF + f, a0, true);
-                        cur = sDst[CH * c + p];
+                        for (int rr = cur + 1; rr < r; ++rr) store_if(A.H + (int64_t)rr * FF + f, 0.0f, true);
+                        cur = r;
                         hacc = b0;
                         return;
                     }
-                    int dst[CH];
+                    uint32_t rem = m;
+                    int q0 = 0;
+#pragma unroll 1
+                    for (;;) {
+                        const int q1 = rem ? __ffs(rem) - 1 : qend;
 #pragma unroll
-                    for (int q = 0; q < CH; ++q) dst[q] = sDst[CH * c + q];
-#pragma unroll
-                    for (int q = 0; q < CH; ++q) {
-                        const int n = CH * c + q;
-                        const bool st = (m >> q) & 1u;
-                        if (FAST) {
-                            store_if(A.H + (int64_t)cur * FF + f, hacc, st);
-                            hacc = st ? 0.0f : hacc;
-                            cur = st ? dst[q] : cur;
-                            hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
-                        } else if (n < ne) {
-                            if (st) {   // first edge of row dst[q]; rows in between have no edges
-                                store_if(A.H + (int64_t)cur * FF + f, hacc, true);
-                                for (int r = cur + 1; r < dst[q]; ++r) store_if(A.H + (int64_t)r * FF + f, 0.0f, true);
-                                hacc = 0.0f;
-                                cur = dst[q];
-                            }
-                            hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
-                        }
+                        for (int q = 0; q < CH; ++q)
+                            if (q >= q0 && q < q1) hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
+                        if (!rem) break;
+                        const int r = sDst[CH * c + q1];
+                        store_if(A.H + (int64_t)cur * FF + f, hacc, true);
+                        for (int rr = cur + 1; rr < r; ++rr) store_if(A.H + (int64_t)rr * FF + f, 0.0f, true);
+                        hacc = 0.0f;
+                        cur = r;
+                        rem &= rem - 1u;
+                        q0 = q1;
                     }
                 };
-                if (fast) {
 #pragma unroll 1
-                    for (int c = 0; c < TE / CH; ++c) chunk(c, std::true_type{});
-                } else {
-#pragma unroll 1
-                    for (int c = 0; c < TE / CH; ++c)
-                        if (CH * c < ne) chunk(c, std::false_type{});
-                }
+                for (int c = 0; c < TE / CH; ++c)
+                    if (CH * c < ne) chunk(c);
                 tc_fence_before();
                 mbar_arrive(bar(WB_FREE, s));
             }
