@@ -97,19 +97,23 @@ __device__ __forceinline__ void drain_cta(uint32_t mbar, uint32_t &phase, int *d
     wait_mma_cta(mbar, phase, d_err, WAIT_BOUND);
 }
 
-// value(a) for atoms [32g, 32g + 32) of the tile at column f, into the activation tile (zero
-// past N)
+// get(q) for atoms 32 g + q (q < nv) of the tile at column f, into the activation tile (zero
+// for q >= nv, past the last atom)
 template <bool SPLIT, typename Get>
-__device__ __forceinline__ void tile_from(unsigned char *T, int f, int g, int64_t a0, int64_t N, Get get)
+__device__ __forceinline__ void tile_from(unsigned char *T, int f, int g, int nv, Get get)
 {
     using S = NodeSmem<SPLIT>;
     float v[32];
 #pragma unroll
-    for (int q = 0; q < 32; ++q) {
-        const int64_t a = a0 + 32 * g + q;
-        v[q] = a < N ? get(a) : 0.0f;
-    }
+    for (int q = 0; q < 32; ++q) v[q] = q < nv ? get(q) : 0.0f;
     store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * g, v);
+}
+
+// atoms of the tile starting at a0 that column chunk c (32 atoms) holds: min(32, N - a0 - 32 c)
+__device__ __forceinline__ int chunk_atoms(int64_t a0, int c, int64_t N)
+{
+    const int64_t r = N - a0 - 32 * c;
+    return r <= 0 ? 0 : (r >= 32 ? 32 : (int)r);
 }
 
 __device__ __forceinline__ const float *x_row(const NodeTcArgs &A, int t, int64_t a)
@@ -176,36 +180,34 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
         unsigned char *T = sm + S::T;
         bool ok = true;
         for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-            const int64_t a0 = tile * TA;
-            tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.H[a * FF + f]; });
+            const int64_t a0 = tile * TA, ab = a0 + 32 * c;   // this thread's atoms: ab + q, q < nv
+            const int nv = chunk_atoms(a0, c, A.N);
+            const float *Hp = A.H + ab * FF + f;
+            float *Pp = A.P + ((int64_t)A.t * A.N + ab) * FF + f;
+            float *Xp = A.X + ((int64_t)A.t * A.N + ab) * FF + f;
+            tile_from<SPLIT>(T, f, g, nv, [&](int q) { return Hp[q * FF]; });
+            float xr[32];   // the residual's x^t, loaded while the GEMMs run
+#pragma unroll
+            for (int q = 0; q < 32; ++q) xr[q] = q < nv ? ldnc_keep(x_row(A, A.t, ab + q) + f) : 0.0f;
             if (!(ok = gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
-                    const int64_t a = a0 + 32 * c + q;
                     v[q] = fmaf(v[q], su1f, c1f);
-                    if (a < A.N) A.P[((int64_t)A.t * A.N + a) * FF + f] = v[q];
+                    if (q < nv) Pp[q * FF] = v[q];
                     v[q] = ssp_fast(v[q]);
                 }
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
-            }
-            float xr[32];   // the residual's x^t, loaded while the second GEMM runs
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const int64_t a = a0 + 32 * c + q;
-                xr[q] = a < A.N ? __ldg(x_row(A, A.t, a) + f) : 0.0f;
             }
             if (!(ok = gemm_step<SPLIT, false>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int64_t a = a0 + 32 * c + q;
-                    if (a < A.N) A.X[((int64_t)A.t * A.N + a) * FF + f] = fmaf(v[q], su2f, xr[q]) + c2f;
-                }
+                for (int q = 0; q < 32; ++q)
+                    if (q < nv) Xp[q * FF] = fmaf(v[q], su2f, xr[q]) + c2f;
             }
             tc_fence_before();
             __syncthreads();
@@ -238,8 +240,10 @@ __global__ void __launch_bounds__(NT, 1) k_node_readout_tc(NodeTcArgs A)
         unsigned char *T = sm + S::T;
         bool ok = true;
         for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-            const int64_t a0 = tile * TA;
-            tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.X[((int64_t)(A.t) * A.N + a) * FF + f]; });
+            const int64_t a0 = tile * TA, ab = a0 + 32 * c;
+            const int nv = chunk_atoms(a0, c, A.N);
+            const float *Xp = A.X + ((int64_t)A.t * A.N + ab) * FF + f;
+            tile_from<SPLIT>(T, f, g, nv, [&](int q) { return Xp[q * FF]; });
             if (!(ok = gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
@@ -267,11 +271,10 @@ __global__ void __launch_bounds__(NT, 1) k_node_readout_tc(NodeTcArgs A)
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
+                float *Bp = A.Xbar + ab * FF + f;
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int64_t a = a0 + 32 * c + q;
-                    if (a < A.N) A.Xbar[a * FF + f] = v[q];
-                }
+                for (int q = 0; q < 32; ++q)
+                    if (q < nv) Bp[q * FF] = v[q];
             }
             tc_fence_before();
             __syncthreads();
@@ -302,29 +305,30 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
         const float su1f = A.su1[f], su2f = A.su2[f];
         bool ok = true;
         for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
-            const int64_t a0 = tile * TA;
-            tile_from<SPLIT>(T, f, g, a0, A.N, [&](int64_t a) { return A.Xbar[a * FF + f] * su2f; });
+            const int64_t a0 = tile * TA, ab = a0 + 32 * c;
+            const int nv = chunk_atoms(a0, c, A.N);
+            const float *Bp = A.Xbar + ab * FF + f;
+            const float *Pp = A.P + ((int64_t)A.t * A.N + ab) * FF + f;
+            tile_from<SPLIT>(T, f, g, nv, [&](int q) { return Bp[q * FF] * su2f; });
+            float pr[32];   // p of this thread's atoms, loaded while the first GEMM runs
+#pragma unroll
+            for (int q = 0; q < 32; ++q) pr[q] = q < nv ? ldnc_keep(Pp + q * FF) : 0.0f;
             if (!(ok = gemm_step<SPLIT, true>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int64_t a = a0 + 32 * c + q;
-                    const float p = a < A.N ? A.P[((int64_t)A.t * A.N + a) * FF + f] : 0.0f;
-                    v[q] *= su1f * sigmoid_fast(p);
-                }
+                for (int q = 0; q < 32; ++q) v[q] *= su1f * sigmoid_fast(pr[q]);
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
             if (!(ok = gemm_step<SPLIT, true>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
+                float *Hp = A.Hbar + ab * FF + f;
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const int64_t a = a0 + 32 * c + q;
-                    if (a < A.N) A.Hbar[a * FF + f] = v[q];
-                }
+                for (int q = 0; q < 32; ++q)
+                    if (q < nv) Hp[q * FF] = v[q];
             }
             tc_fence_before();
             __syncthreads();
