@@ -782,8 +782,9 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
 // One CTA per SM walks the edges of its rows through a ring of NSTG tile stages, each step on
 // its own warps, so that the basis of one tile, the MMAs of another and the activations and
 // gathers of two more run at the same time:
-//   warps 0-7   P  metadata and basis tile bt of tile k, and the source   -> full_b[s]
-//                  rows x_j copied into the stage (16-byte async copies)
+//   warps 0-7   P  metadata and basis tile bt of tile k                  -> full_b[s]
+//                  the source rows x_j copied into the stage (16-byte    -> full_x[s]
+//                  async copies; they land while the MMAs run)
 //   warp  20    M  MMA1 a = W1 bt (after full_b[s])                      -> full_a[s]
 //                  MMA2 w = W2 s  (after full_t[s]), over a's columns    -> full_w[s]
 //   warps 8-15  S  s = ssp(a + b1) from TMEM into the stage's T tile     -> full_t[s]
@@ -796,7 +797,7 @@ constexpr int WS_WARPS = 21;
 constexpr int WS_P = 2 * WGT, WS_S = 2 * WGT;   // producer and activation threads
 constexpr int WS_M_WARP = 20;
 constexpr int WS_THREADS = WS_WARPS * 32;
-enum WsBar { WB_FULL_B = 0, WB_FULL_A, WB_FULL_T, WB_FULL_W, WB_FREE, WB_KINDS };
+enum WsBar { WB_FULL_B = 0, WB_FULL_A, WB_FULL_T, WB_FULL_W, WB_FREE, WB_FULL_X, WB_KINDS };
 
 template <int KP, bool SPLIT, int NSTG>
 struct WsSmem {
@@ -870,7 +871,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
     const uint32_t wmbar = smem_u32(sm + S::WMBAR), drain = smem_u32(sm + S::DRAIN);
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTG; ++s) {
-            mbar_init(bar(WB_FULL_B, s), 2 * WS_P);   // each P thread: stores, then its copies
+            mbar_init(bar(WB_FULL_B, s), WS_P);   // each P thread once its stores are done
+            mbar_init(bar(WB_FULL_X, s), WS_P);   // each P thread once its row copies have landed
             mbar_init(bar(WB_FULL_A, s), 1);
             mbar_init(bar(WB_FULL_T, s), WS_S);
             mbar_init(bar(WB_FULL_W, s), 1);
@@ -931,7 +933,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
 #pragma unroll
                 for (int r = 8 * (t >> 5); r < 8 * (t >> 5) + 8; ++r)
                     if (r < ne) cp_async16(xs + r * FF * 4, xbase0 + sXo[r] + 4 * (t & 31));
-                cp_async_arrive(bar(WB_FULL_B, s));
+                cp_async_arrive(bar(WB_FULL_X, s));
                 if (k + 1 < nt) npos = load_pos(A, nidx);
             }
             asm volatile("cp.async.wait_all;" ::: "memory");
@@ -985,6 +987,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                         atomicOr(A.d_err, ERRBIT_TIMEOUT);
                     }
                     ok = false;
+                } else {
+                    __nanosleep(32);   // nothing ready: leave the issue slots to the other warps
                 }
                 ok = __all_sync(0xffffffffu, ok);
             }
@@ -1033,8 +1037,9 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
             for (int k = 0; k < nt; ++k) {
                 const int s = k % NSTG, ne = min(TE, e1 - (e0 + k * TE));
                 if (!(ok = ws_wait(bar(WB_FULL_W, s), (k / NSTG) & 1, abort, A.d_err, A.wait_limit))) break;
-                // (completed already: P's metadata and the copied source rows are in place)
+                // P's metadata (completed already) and the copied source rows
                 if (!(ok = ws_wait(bar(WB_FULL_B, s), (k / NSTG) & 1, abort, A.d_err, A.wait_limit))) break;
+                if (!(ok = ws_wait(bar(WB_FULL_X, s), (k / NSTG) & 1, abort, A.d_err, A.wait_limit))) break;
                 tc_fence_after();
                 const float *sXs = reinterpret_cast<const float *>(stage(s) + S::XS) + f;
                 const int *sDst = reinterpret_cast<const int *>(stage(s) + S::DST);
@@ -1160,8 +1165,8 @@ int tc_groups_per_cta(bool split) { return groups_for(split); }
 // G * tc_groups_per_cta(split) + 1 entries.
 cudaError_t launch_edge_tc(const EdgeTcArgs &a, int KP, bool split, bool backward, int G, cudaStream_t s)
 {
-    if (KP == 64) return split ? launch_t<64, true, 2, 32>(a, backward, G, s) : launch_t<64, false, 4, 16>(a, backward, G, s);
-    if (KP == 32) return split ? launch_t<32, true, 2, 32>(a, backward, G, s) : launch_t<32, false, 4, 16>(a, backward, G, s);
+    if (KP == 64) return split ? launch_t<64, true, 2, 16>(a, backward, G, s) : launch_t<64, false, 4, 16>(a, backward, G, s);
+    if (KP == 32) return split ? launch_t<32, true, 2, 16>(a, backward, G, s) : launch_t<32, false, 4, 16>(a, backward, G, s);
     return cudaErrorInvalidValue;
 }
 
