@@ -9,7 +9,7 @@
 //
 // Two builders:
 //   * open boundaries (or a box too small for a 3x3x3 cell stencil): all pairs of a replica,
-//     positions staged through shared memory in tiles of 128; sources come out ascending;
+//     positions staged through shared memory in tiles of 512; sources come out ascending;
 //   * periodic boxes with >= 3 cells per axis: cell list (cell side >= r_cut * 1.0001), then
 //     each row is sorted by source.  Atoms are binned by their coordinates wrapped into the
 //     box in double precision.  The fp32 test on raw coordinates can accept a pair whose
@@ -28,7 +28,7 @@ namespace sn {
 
 namespace {
 
-constexpr int BT = 128;   // threads per CTA / positions per shared-memory tile
+constexpr int BT = 128;   // threads per CTA of the cell-list kernels
 
 __device__ __forceinline__ float min_image_axis(float dx, float L)
 {
@@ -67,10 +67,15 @@ __global__ void k_prep_positions(const float *__restrict__ pos, float4 *__restri
 }
 
 // -------------------------------------------------------------------- all pairs per replica
-// One warp per destination atom i: lane l tests sources j = j0 + l of i's replica, a ballot
-// gives the hits in ascending j, and FILL writes them at row_ptr[i] + (hits before it) while
-// the count pass stores their number.  FILL = false counts, true writes sources in ascending
-// order.
+// CTA (b, r) of 8 warps: destination atoms 32 b + [0, 32) of replica r, 4 per warp.  The
+// replica's positions pass through shared memory in tiles of PT; for each of its atoms a warp
+// tests 32 sources per step (lane l: source j0 + l), a ballot gives the hits in ascending j,
+// and FILL writes them at row_ptr[i] + (hits before it) while the count pass stores their
+// number.  Decisions to stop are taken once per CTA (its threads meet at the tile barriers).
+constexpr int PT = 512;            // positions per shared-memory tile
+constexpr int PW = 4;              // destination atoms per warp
+constexpr int PA = 8 * PW;         // destination atoms per CTA
+
 template <bool FILL>
 __global__ void __launch_bounds__(256) k_pairs(const float4 *__restrict__ pos4, int n_per, Geometry g, float rc2,
                                                int32_t *__restrict__ cnt, const int32_t *__restrict__ row_ptr,
@@ -79,34 +84,57 @@ __global__ void __launch_bounds__(256) k_pairs(const float4 *__restrict__ pos4, 
 {
     pdl_trigger();
     pdl_wait();
-    const int64_t i = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (i >= N) return;
-    // (read once per warp: every exit below is taken by the whole warp)
-    const int err = __shfl_sync(0xffffffffu, lane == 0 ? *((volatile int *)d_err) : 0, 0);
-    if (err & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) return;
-    if (FILL && (int64_t)row_ptr[N] > cap) {
-        if (lane == 0) atomicOr(d_err, ERRBIT_CAPACITY);
-        return;
-    }
-    const int64_t base = i / n_per * n_per;
-    const int il = (int)(i - base);
-    const float4 pi = __ldg(pos4 + i);
-    int32_t w = FILL ? row_ptr[i] : 0;
-    bool degenerate = false;
-    for (int j0 = 0; j0 < n_per; j0 += 32) {
-        const int jl = j0 + lane;
-        bool hit = false;
-        if (jl < n_per && jl != il) {
-            const float r2 = pair_r2(pi, __ldg(pos4 + base + jl), g);
-            hit = r2 < rc2;
-            degenerate |= hit && r2 == 0.0f;
+    __shared__ float4 sp[PT];
+    __shared__ int s_stop;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t base = (int64_t)blockIdx.y * n_per;
+    if (threadIdx.x == 0) {
+        int stop = (*((volatile int *)d_err) & (ERRBIT_NONFINITE | ERRBIT_CAPACITY)) != 0;
+        if (FILL && !stop && (int64_t)row_ptr[N] > cap) {
+            atomicOr(d_err, ERRBIT_CAPACITY);
+            stop = 1;
         }
-        const unsigned m = __ballot_sync(0xffffffffu, hit);
-        if (FILL && hit) col[w + __popc(m & ((1u << lane) - 1u))] = (int32_t)(base + jl);
-        w += __popc(m);
+        s_stop = stop;
     }
-    if (!FILL && lane == 0) cnt[i] = w;
+    __syncthreads();
+    if (s_stop) return;
+    const int il0 = blockIdx.x * PA + wid * PW;   // this warp's first atom (index in the replica)
+    float4 pi[PW];
+    int32_t w[PW];
+#pragma unroll
+    for (int a = 0; a < PW; ++a) {
+        const bool valid = il0 + a < n_per;
+        pi[a] = valid ? __ldg(pos4 + base + il0 + a) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        w[a] = FILL && valid ? row_ptr[base + il0 + a] : 0;
+    }
+    bool degenerate = false;
+    for (int t0 = 0; t0 < n_per; t0 += PT) {
+        const int tn = min(PT, n_per - t0);
+        __syncthreads();   // the previous tile is read
+        for (int q = threadIdx.x; q < tn; q += 256) sp[q] = __ldg(pos4 + base + t0 + q);
+        __syncthreads();
+#pragma unroll
+        for (int a = 0; a < PW; ++a) {
+            if (il0 + a >= n_per) continue;   // (warp-uniform)
+            for (int j0 = 0; j0 < tn; j0 += 32) {
+                const int jl = j0 + lane, j = t0 + jl;
+                bool hit = false;
+                if (jl < tn && j != il0 + a) {
+                    const float r2 = pair_r2(pi[a], sp[jl], g);
+                    hit = r2 < rc2;
+                    degenerate |= hit && r2 == 0.0f;
+                }
+                const unsigned m = __ballot_sync(0xffffffffu, hit);
+                if (FILL && hit) col[w[a] + __popc(m & ((1u << lane) - 1u))] = (int32_t)(base + j);
+                w[a] += __popc(m);
+            }
+        }
+    }
+    if (!FILL && lane == 0) {
+#pragma unroll
+        for (int a = 0; a < PW; ++a)
+            if (il0 + a < n_per) cnt[base + il0 + a] = w[a];
+    }
     if (FILL && __any_sync(0xffffffffu, degenerate) && lane == 0) atomicOr(d_err, ERRBIT_DEGENERATE);
 }
 
@@ -430,8 +458,8 @@ cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *po
         trace_end(tr, s);
     } else {
         trace_begin(tr, KK_NB_COUNT, s);
-        if ((e = launch_pdl(k_pairs<false>, dim3(blocks_for(32 * N, 256)), dim3(256), 0, s, pos4, sys.n_per_replica, g,
-                            rc2, w.cnt, row_ptr, col, cap, N, d_err)))
+        if ((e = launch_pdl(k_pairs<false>, dim3(blocks_for(sys.n_per_replica, PA), sys.n_replicas), dim3(256), 0, s,
+                            pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col, cap, N, d_err)))
             return e;
         trace_end(tr, s);
     }
@@ -452,8 +480,8 @@ cudaError_t launch_neighbors(const sn_system &sys, float r_cut, const float4 *po
                             w.cell_start, w.cell_atoms, w.cnt, row_ptr, col, cap, d_err)))
             return e;
     } else {
-        if ((e = launch_pdl(k_pairs<true>, dim3(blocks_for(32 * N, 256)), dim3(256), 0, s, pos4, sys.n_per_replica, g,
-                            rc2, w.cnt, row_ptr, col, cap, N, d_err)))
+        if ((e = launch_pdl(k_pairs<true>, dim3(blocks_for(sys.n_per_replica, PA), sys.n_replicas), dim3(256), 0, s,
+                            pos4, sys.n_per_replica, g, rc2, w.cnt, row_ptr, col, cap, N, d_err)))
             return e;
     }
     trace_end(tr, s);
