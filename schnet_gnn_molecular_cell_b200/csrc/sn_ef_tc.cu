@@ -782,19 +782,23 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
 // One CTA per SM walks the edges of its rows through a ring of NSTG tile stages, each step on
 // its own warps, so that the basis of one tile, the MMAs of another and the activations and
 // gathers of two more run at the same time:
-//   warps 0-7   P  metadata and basis tile bt of tile k                  -> full_b[s]
+//   warps 12-19 P  metadata and basis tile bt of tile k                  -> full_b[s]
 //                  the source rows x_j copied into the stage (16-byte    -> full_x[s]
 //                  async copies; they land while the MMAs run)
 //   warp  20    M  MMA1 a = W1 bt (after full_b[s])                      -> full_a[s]
 //                  MMA2 w = W2 s  (after full_t[s]), over a's columns    -> full_w[s]
-//   warps 8-15  S  s = ssp(a + b1) from TMEM into the stage's T tile     -> full_t[s]
+//   warps 4-11  S  s = ssp(a + b1) from TMEM into the stage's T tile     -> full_t[s]
 //                  (two warpgroups, 32 of the tile's 64 columns each)
-//   warps 16-19 E  h_i += x_j (.) (w + b2), running sums per row         -> free[s]
+//   warps 0-3   E  h_i += x_j (.) (w + b2), running sums per row         -> free[s]
 // Stage s = k % NSTG holds the tile's basis and activation tiles, its metadata, the source
 // rows x_j and 64 TMEM columns.  Each barrier of stage s completes once per tile using the stage, so tile k waits
 // for parity (k / NSTG) & 1 (and P, before refilling the stage, for the previous use's free).
 constexpr int WS_WARPS = 21;
 constexpr int WS_P = 2 * WGT, WS_S = 2 * WGT;   // producer and activation threads
+// Roles by warp: E 0-3, S 4-11, P 12-19, M 20.  The epilogue, the ring's longest stage, takes
+// the lowest warp indices: when several warps of a scheduler can issue, the older (lower)
+// warps tend to be picked, and the producer and activation warps have slack to give.
+constexpr int WS_E_WARP0 = 0, WS_S_WARP0 = 4, WS_P_WARP0 = 12;
 constexpr int WS_M_WARP = 20;
 constexpr int WS_THREADS = WS_WARPS * 32;
 enum WsBar { WB_FULL_B = 0, WB_FULL_A, WB_FULL_T, WB_FULL_W, WB_FREE, WB_FULL_X, WB_KINDS };
@@ -908,10 +912,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
     const int e0 = r0 < r1 ? A.row_ptr[r0] : 0, e1 = r0 < r1 ? A.row_ptr[r1] : 0;
     const int nt = (e1 - e0 + TE - 1) / TE;
     if (!skip && r0 < r1) {
-        if (warp < 8) {
+        if (warp >= WS_P_WARP0 && warp < WS_M_WARP) {
             // P: the prologue of tile k (edge n = t % 64, a quarter of its Gaussians per
             // thread), with tile k + 1's indices and positions read ahead
-            const int t = threadIdx.x, nf = t & (TE - 1);
+            const int t = threadIdx.x - 32 * WS_P_WARP0, nf = t & (TE - 1);
             EdgeIdx nidx = load_idx(A, e0 + nf, e1);
             EdgePos npos = load_pos(A, nidx);
             const float *xbase0 = x_base(A, 0);
@@ -1003,9 +1007,9 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                     }
                 __syncwarp();
             }
-        } else if (warp < 16) {
+        } else if (warp >= WS_S_WARP0) {
             // S: s = ssp(a + b1) into the stage's activation tile, columns [32 sg, 32 sg + 32)
-            const int f = (threadIdx.x - WS_P) % WGT, sg = (threadIdx.x - WS_P) / WGT;
+            const int f = (threadIdx.x - 32 * WS_S_WARP0) % WGT, sg = (threadIdx.x - 32 * WS_S_WARP0) / WGT;
             const float b1f = A.b1[f], s1f = A.s1[f];
             const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
             for (int k = 0; k < nt; ++k) {
@@ -1028,7 +1032,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
         } else {
             // E: h_i += x_src (.) (w + b2); a row is written when the next one starts (rows in
             // between, and after the last edge, have no edges and receive zero)
-            const int f = threadIdx.x - WS_P - WS_S;
+            const int f = threadIdx.x - 32 * WS_E_WARP0;
             const float b2f = A.b2[f], s2f = A.s2[f];
             const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
             int cur = r0;
