@@ -67,8 +67,7 @@ struct TcSmem {
     static constexpr uint32_t FV = UVEC + 12 * TE;      // float[TE][3]
     static constexpr uint32_t MASK = FV + 12 * TE;      // uint32[4]: row starts, empty-row flags
     static constexpr uint32_t CD = MASK + 16;           // float2[TE]: C(d), dC/dd (fp16 backward)
-    static constexpr uint32_t TDST = CD + 8 * TE;       // int[TE]: type of the destination (block 0)
-    static constexpr uint32_t PDX = TDST + 4 * TE;      // float[4]: force scan, warp 0 -> warp 1
+    static constexpr uint32_t PDX = CD + 8 * TE;        // float[4]: force scan, warp 0 -> warp 1
     static constexpr uint32_t MBAR = PDX + 16;          // uint64
     static constexpr uint32_t REGION = (MBAR + 8 + 127) / 128 * 128;
     static constexpr uint32_t HOLD = GROUPS + NW * REGION;
@@ -93,7 +92,6 @@ struct EdgePos {
     float4 ri, rj;
     int tj, rs;   // type of the source (block 0), first edge of the destination's row
     int rsm;      // first edge of the row before the destination's (-1 for row 0)
-    int ti;       // type of the destination (block 0)
 };
 
 // (loads kept where they stand, so that the read-ahead by a tile really is ahead: see ld_keep)
@@ -115,7 +113,6 @@ __device__ __forceinline__ EdgePos load_pos(const EdgeTcArgs &A, EdgeIdx x)
     p.tj = A.t == 0 ? ldnc_keep(A.types + x.j) : 0;
     p.rs = ldnc_keep(A.row_ptr + x.i);
     p.rsm = x.i > 0 ? ldnc_keep(A.row_ptr + x.i - 1) : -1;
-    p.ti = A.t == 0 ? ldnc_keep(A.types + x.i) : 0;
     return p;
 }
 
@@ -140,7 +137,7 @@ __device__ __forceinline__ const float *x_row(const EdgeTcArgs &A, const float *
 // SHARED (fp16, warp-specialised producer): part 0 alone forms d and C(d) and leaves them in
 // the stage (S::DF, S::CC) for the other parts, after a barrier over the 64 PARTS threads.
 // STORE_CD (fp16 backward): part 0 also leaves C(d) and dC/dd of every edge in the stage
-// (S::CD, float2[TE]) for the dbar step, and the destination's type (S::TDST, int[TE], block 0).
+// (S::CD, float2[TE]) for the dbar step.
 template <class S, int KP, bool SPLIT, bool BWD, int PARTS = 2, bool SHARED = false, bool STORE_CD = false>
 __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigned char *sm, unsigned char *R, int t,
                                               int ts, int ne, EdgeIdx x, const EdgePos &p)
@@ -166,7 +163,6 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
         d = sqrt(dx * dx + dy * dy + dz * dz);
         if (half == 0) {
             sDst[n] = i;
-            if constexpr (STORE_CD) reinterpret_cast<int *>(R + S::TDST)[n] = p.ti;
             sDist[n] = (double)d;
             const real inv = (real)1 / d;
             sU[3 * n] = (float)(dx * inv);
@@ -178,7 +174,6 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
         }
     } else if (half == 0) {
         sDst[n] = -1;
-        if constexpr (STORE_CD) reinterpret_cast<int *>(R + S::TDST)[n] = 0;
         sDist[n] = 0.0;
     } else if (half == 1) {
         if (BWD) reinterpret_cast<int2 *>(sXo)[n] = make_int2(0, 0);
@@ -800,6 +795,8 @@ constexpr int WS_P = 2 * WGT, WS_S = 2 * WGT;   // producer and activation threa
 // warps tend to be picked, and the producer and activation warps have slack to give.
 constexpr int WS_E_WARP0 = 0, WS_S_WARP0 = 4, WS_P_WARP0 = 12;
 constexpr int WS_M_WARP = 20;
+constexpr int WS_CH = 8;   // TMEM columns (edges) per chunk of the activation warps
+constexpr int WS_CE = 8;   // and of the epilogue warps
 constexpr int WS_THREADS = WS_WARPS * 32;
 enum WsBar { WB_FULL_B = 0, WB_FULL_A, WB_FULL_T, WB_FULL_W, WB_FREE, WB_FULL_X, WB_KINDS };
 
@@ -862,7 +859,7 @@ static __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, vo
     return __all_sync(0xffffffffu, ok) != 0;
 }
 
-template <int KP, bool SPLIT, int NSTG, int CH>
+template <int KP, bool SPLIT, int NSTG, int CH, int CE>
 __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int parts_per_cta)
 {
     using S = WsSmem<KP, SPLIT, NSTG>;
@@ -1054,30 +1051,30 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                 // finished row is written when the next starts, rows in between (without edges)
                 // receive zero
                 auto chunk = [&](int c) {
-                    float v[CH], xs[CH];
-                    tmem_ld<CH>(tmem + lanes + 64 * s + CH * c, v);
+                    float v[CE], xs[CE];
+                    tmem_ld<CE>(tmem + lanes + 64 * s + CE * c, v);
 #pragma unroll
-                    for (int q = 0; q < CH; ++q) xs[q] = sXs[(CH * c + q) * FF];
-                    const uint32_t m = (uint32_t)(starts >> (CH * c)) & (CH >= 32 ? 0xffffffffu : (1u << (CH & 31)) - 1u);
-                    const int qend = min(CH, ne - CH * c);   // valid edges of the chunk (>= 1)
-                    if (qend == CH && m == 0) {   // the chunk continues the current row
+                    for (int q = 0; q < CE; ++q) xs[q] = sXs[(CE * c + q) * FF];
+                    const uint32_t m = (uint32_t)(starts >> (CE * c)) & (CE >= 32 ? 0xffffffffu : (1u << (CE & 31)) - 1u);
+                    const int qend = min(CE, ne - CE * c);   // valid edges of the chunk (>= 1)
+                    if (qend == CE && m == 0) {   // the chunk continues the current row
 #pragma unroll
-                        for (int q = 0; q < CH; ++q) hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
+                        for (int q = 0; q < CE; ++q) hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
                         return;
                     }
-                    if (qend == CH && (m & (m - 1u)) == 0) {
+                    if (qend == CE && (m & (m - 1u)) == 0) {
                         // one row starts at edge p of the chunk: edges before it finish row cur,
                         // edges from it open the next row (two running sums, one pass)
                         const int p = __ffs(m) - 1;
                         float a0 = hacc, b0 = 0.0f;
 #pragma unroll
-                        for (int q = 0; q < CH; ++q) {
+                        for (int q = 0; q < CE; ++q) {
                             const bool before = q < p;
                             const float t0 = fmaf(xs[q], fmaf(v[q], s2f, b2f), before ? a0 : b0);
                             a0 = before ? t0 : a0;
                             b0 = before ? b0 : t0;
                         }
-                        const int r = sDst[CH * c + p];
+                        const int r = sDst[CE * c + p];
                         store_if(A.H + (int64_t)cur * FF + f, a0, true);
                         for (int rr = cur + 1; rr < r; ++rr) store_if(A.H + (int64_t)rr * FF + f, 0.0f, true);
                         cur = r;
@@ -1090,10 +1087,10 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                     for (;;) {
                         const int q1 = rem ? __ffs(rem) - 1 : qend;
 #pragma unroll
-                        for (int q = 0; q < CH; ++q)
+                        for (int q = 0; q < CE; ++q)
                             if (q >= q0 && q < q1) hacc = fmaf(xs[q], fmaf(v[q], s2f, b2f), hacc);
                         if (!rem) break;
-                        const int r = sDst[CH * c + q1];
+                        const int r = sDst[CE * c + q1];
                         store_if(A.H + (int64_t)cur * FF + f, hacc, true);
                         for (int rr = cur + 1; rr < r; ++rr) store_if(A.H + (int64_t)rr * FF + f, 0.0f, true);
                         hacc = 0.0f;
@@ -1103,8 +1100,8 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                     }
                 };
 #pragma unroll 1
-                for (int c = 0; c < TE / CH; ++c)
-                    if (CH * c < ne) chunk(c);
+                for (int c = 0; c < TE / CE; ++c)
+                    if (CE * c < ne) chunk(c);
                 tc_fence_before();
                 mbar_arrive(bar(WB_FREE, s));
             }
@@ -1147,8 +1144,8 @@ cudaError_t launch_t(const EdgeTcArgs &a, bool backward, int G, cudaStream_t s)
         constexpr int NSTG = 3;
         using WS = WsSmem<KP, false, NSTG>;
         static_assert(WS::BYTES <= 227 * 1024, "shared memory plan exceeds 227 KB");
-        if ((e = prepare(k_edge_fwd_ws<KP, false, NSTG, CH>, WS::BYTES))) return e;
-        e = launch_pdl(k_edge_fwd_ws<KP, false, NSTG, CH>, dim3(G), dim3(WS_THREADS), WS::BYTES, s, a, NW);
+        if ((e = prepare(k_edge_fwd_ws<KP, false, NSTG, WS_CH, WS_CE>, WS::BYTES))) return e;
+        e = launch_pdl(k_edge_fwd_ws<KP, false, NSTG, WS_CH, WS_CE>, dim3(G), dim3(WS_THREADS), WS::BYTES, s, a, NW);
     } else {
         if ((e = prepare(k_edge_fwd_tc<KP, SPLIT, NW, CH>, S::BYTES))) return e;
         e = launch_pdl(k_edge_fwd_tc<KP, SPLIT, NW, CH>, dim3(G), dim3(WGT * NW), S::BYTES, s, a);
