@@ -153,7 +153,9 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
     // (double for the fp32-accurate split mode, float for fp16 operands)
     using real = typename std::conditional<SPLIT, double, float>::type;
     real d = 0;
-    if (n < ne && (!SHARED || half <= 1)) {
+    // (SHARED: the source rows are copied by offsets the producer holds, so only part 0 works
+    // here; the distance and direction arrays serve the backward's forces only)
+    if (n < ne && (SHARED ? half == 0 : half <= 1)) {
         const int i = x.i, j = x.j;
         const float4 ri = p.ri, rj = p.rj;
         real dx = (real)ri.x - (real)rj.x, dy = (real)ri.y - (real)rj.y, dz = (real)ri.z - (real)rj.z;
@@ -163,19 +165,21 @@ __device__ __forceinline__ void tile_prologue(const EdgeTcArgs &A, const unsigne
         d = sqrt(dx * dx + dy * dy + dz * dz);
         if (half == 0) {
             sDst[n] = i;
-            sDist[n] = (double)d;
-            const real inv = (real)1 / d;
-            sU[3 * n] = (float)(dx * inv);
-            sU[3 * n + 1] = (float)(dy * inv);
-            sU[3 * n + 2] = (float)(dz * inv);
+            if constexpr (BWD) {
+                sDist[n] = (double)d;
+                const real inv = (real)1 / d;
+                sU[3 * n] = (float)(dx * inv);
+                sU[3 * n + 1] = (float)(dy * inv);
+                sU[3 * n + 2] = (float)(dz * inv);
+            }
         } else if (half == 1) {
             if (BWD) reinterpret_cast<int2 *>(sXo)[n] = make_int2((A.t == 0 ? p.tj : j) * FF, j * FF);
             else sXo[n] = (A.t == 0 ? p.tj : j) * FF;
         }
     } else if (half == 0) {
         sDst[n] = -1;
-        sDist[n] = 0.0;
-    } else if (half == 1) {
+        if constexpr (BWD) sDist[n] = 0.0;
+    } else if (half == 1 && !SHARED) {
         if (BWD) reinterpret_cast<int2 *>(sXo)[n] = make_int2(0, 0);
         else sXo[n] = 0;
     }
@@ -777,9 +781,10 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
 // One CTA per SM walks the edges of its rows through a ring of NSTG tile stages, each step on
 // its own warps, so that the basis of one tile, the MMAs of another and the activations and
 // gathers of two more run at the same time:
-//   warps 12-19 P  metadata and basis tile bt of tile k                  -> full_b[s]
-//                  the source rows x_j copied into the stage (16-byte    -> full_x[s]
-//                  async copies; they land while the MMAs run)
+//   warps 12-19 P  the source rows x_j copied into the stage (16-byte    -> full_x[s]
+//                  async copies, issued first; they land while the
+//                  prologue and the MMAs run)
+//                  metadata and basis tile bt of tile k                  -> full_b[s]
 //   warp  20    M  MMA1 a = W1 bt (after full_b[s])                      -> full_a[s]
 //                  MMA2 w = W2 s  (after full_t[s]), over a's columns    -> full_w[s]
 //   warps 4-11  S  s = ssp(a + b1) from TMEM into the stage's T tile     -> full_t[s]
@@ -924,17 +929,24 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                 const EdgeIdx cidx = nidx;
                 const EdgePos cpos = npos;
                 if (k + 1 < nt) nidx = load_idx(A, ts + TE + nf, e1);
+                {
+                    // source rows first, so that they land during the prologue: warp w holds
+                    // edges 32 (w % 2) + lane and copies eight of them, 32 (w % 2) + 8 (w / 2) + i,
+                    // lane l their bytes [16 l, 16 l + 16), the row offsets passed by shuffles
+                    const int w = t >> 5, lane = t & 31;
+                    const int off = (A.t == 0 ? cpos.tj : cidx.j) * FF;
+                    const uint32_t xs = smem_u32(stage(s) + S::XS) + 16 * lane;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int src = 8 * (w >> 1) + i, r = 32 * (w & 1) + src;
+                        const int o = __shfl_sync(0xffffffffu, off, src);
+                        if (r < ne) cp_async16(xs + r * FF * 4, xbase0 + o + 4 * lane);
+                    }
+                    cp_async_arrive(bar(WB_FULL_X, s));
+                }
                 tile_prologue<S, KP, SPLIT, false, 4, true>(A, sm, stage(s), t, ts, ne, cidx, cpos);
                 fence_async_smem();
                 mbar_arrive(bar(WB_FULL_B, s));
-                named_sync(5, WS_P);   // every edge's gather offset is in shared memory
-                // source rows: warp w copies rows 8w .. 8w + 7, lane l their bytes [16 l, 16 l + 16)
-                const int *sXo = reinterpret_cast<const int *>(stage(s) + S::XO);
-                const uint32_t xs = smem_u32(stage(s) + S::XS) + 16 * (t & 31);
-#pragma unroll
-                for (int r = 8 * (t >> 5); r < 8 * (t >> 5) + 8; ++r)
-                    if (r < ne) cp_async16(xs + r * FF * 4, xbase0 + sXo[r] + 4 * (t & 31));
-                cp_async_arrive(bar(WB_FULL_X, s));
                 if (k + 1 < nt) npos = load_pos(A, nidx);
             }
             asm volatile("cp.async.wait_all;" ::: "memory");
