@@ -603,9 +603,10 @@ __global__ void k_partition_rows(const int32_t *__restrict__ row_ptr, int64_t N,
     for (int32_t e = e0 + lane; e < e1; e += 32) dst[e] = (int32_t)i;
 }
 
-EdgeTcArgs tc_args(const EdgeArgs &a, const BlockW &bw, int *d_err, long long wait_limit)
+EdgeTcArgs tc_args(const EdgeArgs &a, const BlockW &bw, int n_types, int *d_err, long long wait_limit)
 {
     EdgeTcArgs t{};
+    t.n_types = n_types;
     t.wait_limit = wait_limit;
     t.pos4 = a.pos4;
     t.types = a.types;
@@ -745,7 +746,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
             ea.w = m.blk[t];
             ea.t = t;
             trace_begin(tr, KK_EDGE_FWD, s);
-            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err, w.wait_limit), KP, split, false, w.G, s))) return e;
+            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], m.n_types, d_err, w.wait_limit), KP, split, false, w.G, s))) return e;
             trace_end(tr, s);
             trace_begin(tr, KK_NODE_FWD, s);
             if ((e = launch_node_tc(node_args(t), split, 0, n_sm, s))) return e;
@@ -761,7 +762,7 @@ cudaError_t run(const Model &m, const sn_system &sys, const Geometry &geo, const
             ea.w = m.blk[t];
             ea.t = t;
             trace_begin(tr, KK_EDGE_BWD, s);
-            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], d_err, w.wait_limit), KP, split, true, w.G, s))) return e;
+            if ((e = launch_edge_tc(tc_args(ea, m.blk[t], m.n_types, d_err, w.wait_limit), KP, split, true, w.G, s))) return e;
             trace_end(tr, s);
         }
         return cudaGetLastError();

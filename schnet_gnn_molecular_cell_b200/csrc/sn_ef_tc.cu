@@ -24,6 +24,8 @@
 //   (r % 8) * 16 + (r / 8) * SBO + (c % 8) * 2 + (c / 8) * LBO   bytes.
 // The same bytes read as K-major for one GEMM read as MN-major for its transpose with LBO and
 // SBO exchanged, so each weight matrix is stored once and serves forward and backward.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -781,9 +783,10 @@ __global__ void __launch_bounds__(WGT *NW, 1) k_edge_bwd_tc(EdgeTcArgs A)
 // One CTA per SM walks the edges of its rows through a ring of NSTG tile stages, each step on
 // its own warps, so that the basis of one tile, the MMAs of another and the activations and
 // gathers of two more run at the same time:
-//   warps 12-19 P  the source rows x_j copied into the stage (16-byte    -> full_x[s]
-//                  async copies, issued first; they land while the
-//                  prologue and the MMAs run)
+//   warps 12-19 P  the source rows x_j gathered into the stage by the    -> full_x[s]
+//                  tensor memory accelerator (four rows per instruction,
+//                  issued first; they land while the prologue and the
+//                  MMAs run)
 //                  metadata and basis tile bt of tile k                  -> full_b[s]
 //   warp  20    M  MMA1 a = W1 bt (after full_b[s])                      -> full_a[s]
 //                  MMA2 w = W2 s  (after full_t[s]), over a's columns    -> full_w[s]
@@ -835,9 +838,11 @@ struct WsSmem {
     static constexpr uint32_t DRAIN = WMBAR + 8;                   // last MMAs before teardown
     static constexpr uint32_t HOLD = DRAIN + 8;                    // TMEM address
     static constexpr uint32_t ABORT = HOLD + 8;                    // int: a wait timed out
+    static constexpr uint32_t SKIP = ABORT + 4;                    // int: an earlier kernel failed
     static constexpr uint32_t MUH = ABORT + 8;
     static constexpr uint32_t MUL = MUH + 256;
     static constexpr uint32_t BYTES = MUL + 256;
+    static constexpr uint32_t ALLOC = BYTES + 128;   // with the slack to align the base to 128 bytes
     static constexpr uint32_t TMEM_COLS = NSTG * 64 <= 128 ? 128 : NSTG * 64 <= 256 ? 256 : 512;
 };
 
@@ -864,12 +869,18 @@ static __device__ __forceinline__ bool ws_wait(uint32_t bar, uint32_t parity, vo
     return __all_sync(0xffffffffu, ok) != 0;
 }
 
+// xmap: the block's source feature rows (x^t, or the embedding table in block 0) as a 2-D
+// tensor [rows][F] of fp32 with boxes of one row.  The shared-memory plan starts at the first
+// 128-byte boundary of the dynamic window, so that the stages' row tiles, the gathers'
+// destinations, are 128-byte aligned.
 template <int KP, bool SPLIT, int NSTG, int CH, int CE>
-__global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int parts_per_cta)
+__global__ void __launch_bounds__(WS_THREADS, 1)
+    k_edge_fwd_ws(EdgeTcArgs A, int parts_per_cta, const __grid_constant__ CUtensorMap xmap)
 {
     using S = WsSmem<KP, SPLIT, NSTG>;
-    extern __shared__ __align__(128) unsigned char sm[];
-    __shared__ int skip;
+    extern __shared__ __align__(128) unsigned char sm_window[];
+    unsigned char *const sm = sm_window + ((128u - (smem_u32(sm_window) & 127u)) & 127u);
+    int &skip = *reinterpret_cast<int *>(sm + S::SKIP);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     auto bar = [&](int kind, int s) { return smem_u32(sm + S::BARS + 8 * (kind * NSTG + s)); };
     auto stage = [&](int s) { return sm + S::STAGES + s * S::STG; };
@@ -878,7 +889,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTG; ++s) {
             mbar_init(bar(WB_FULL_B, s), WS_P);   // each P thread once its stores are done
-            mbar_init(bar(WB_FULL_X, s), WS_P);   // each P thread once its row copies have landed
+            mbar_init(bar(WB_FULL_X, s), 2);      // P warps 0 and 1, with the bytes of their gathers
             mbar_init(bar(WB_FULL_A, s), 1);
             mbar_init(bar(WB_FULL_T, s), WS_S);
             mbar_init(bar(WB_FULL_W, s), 1);
@@ -920,7 +931,6 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
             const int t = threadIdx.x - 32 * WS_P_WARP0, nf = t & (TE - 1);
             EdgeIdx nidx = load_idx(A, e0 + nf, e1);
             EdgePos npos = load_pos(A, nidx);
-            const float *xbase0 = x_base(A, 0);
             for (int k = 0; k < nt; ++k) {
                 const int s = k % NSTG, ts = e0 + k * TE, ne = min(TE, e1 - ts);
                 int okw = 1;
@@ -929,27 +939,28 @@ __global__ void __launch_bounds__(WS_THREADS, 1) k_edge_fwd_ws(EdgeTcArgs A, int
                 const EdgeIdx cidx = nidx;
                 const EdgePos cpos = npos;
                 if (k + 1 < nt) nidx = load_idx(A, ts + TE + nf, e1);
-                {
-                    // source rows first, so that they land during the prologue: warp w holds
-                    // edges 32 (w % 2) + lane and copies eight of them, 32 (w % 2) + 8 (w / 2) + i,
-                    // lane l their bytes [16 l, 16 l + 16), the row offsets passed by shuffles
+                if (t < 64) {
+                    // source rows first, so that they land during the prologue: lane 4 g of P
+                    // warp w (0 or 1) gathers the rows of edges 32 w + 4 g + [0, 4), which lanes
+                    // 4 g .. 4 g + 3 hold (padding edges of the last group read the row of atom 0);
+                    // lane 0 first announces the warp's bytes on the stage's barrier
                     const int w = t >> 5, lane = t & 31;
-                    const int off = (A.t == 0 ? cpos.tj : cidx.j) * FF;
-                    const uint32_t xs = smem_u32(stage(s) + S::XS) + 16 * lane;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int src = 8 * (w >> 1) + i, r = 32 * (w & 1) + src;
-                        const int o = __shfl_sync(0xffffffffu, off, src);
-                        if (r < ne) cp_async16(xs + r * FF * 4, xbase0 + o + 4 * lane);
-                    }
-                    cp_async_arrive(bar(WB_FULL_X, s));
+                    const int row = A.t == 0 ? cpos.tj : cidx.j;
+                    const int r1 = __shfl_down_sync(0xffffffffu, row, 1);
+                    const int r2 = __shfl_down_sync(0xffffffffu, row, 2);
+                    const int r3 = __shfl_down_sync(0xffffffffu, row, 3);
+                    const int groups = min(8, max(0, (ne - 32 * w + 3) / 4));
+                    if (lane == 0) mbar_expect_tx(bar(WB_FULL_X, s), (uint32_t)groups * 4 * FF * 4);
+                    __syncwarp();
+                    if ((lane & 3) == 0 && (lane >> 2) < groups)
+                        tma_gather4(smem_u32(stage(s) + S::XS) + (32 * w + lane) * FF * 4, &xmap, 0, row, r1, r2, r3,
+                                    bar(WB_FULL_X, s));
                 }
                 tile_prologue<S, KP, SPLIT, false, 4, true>(A, sm, stage(s), t, ts, ne, cidx, cpos);
                 fence_async_smem();
                 mbar_arrive(bar(WB_FULL_B, s));
                 if (k + 1 < nt) npos = load_pos(A, nidx);
             }
-            asm volatile("cp.async.wait_all;" ::: "memory");
         } else if (warp == WS_M_WARP) {
             // M: lane 0 polls the two queues and issues whichever MMA is ready: MMA1 of the next
             // tile whose basis is in (and whose stage E has released), MMA2 of the oldest tile
@@ -1142,6 +1153,30 @@ cudaError_t prepare(Kern k, uint32_t bytes)
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// Tensor map of rows x [0, rows) of an fp32 matrix [rows][F] at base (256-byte aligned): boxes
+// of one row (F elements), no swizzle, zero fill outside, for the four-row gathers.
+cudaError_t make_row_map(CUtensorMap *map, const float *base, int64_t rows)
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || !fn) return cudaErrorNotSupported;
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (rows < 1 || rows > (1ll << 31)) return cudaErrorInvalidValue;
+    const cuuint64_t dims[2] = {(cuuint64_t)FF, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)FF * sizeof(float)};
+    const cuuint32_t box[2] = {(cuuint32_t)FF, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(base), dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int KP, bool SPLIT, int NW, int CH>
 cudaError_t launch_t(const EdgeTcArgs &a, bool backward, int G, cudaStream_t s)
 {
@@ -1155,9 +1190,14 @@ cudaError_t launch_t(const EdgeTcArgs &a, bool backward, int G, cudaStream_t s)
     } else if constexpr (!SPLIT) {
         constexpr int NSTG = 3;
         using WS = WsSmem<KP, false, NSTG>;
-        static_assert(WS::BYTES <= 227 * 1024, "shared memory plan exceeds 227 KB");
-        if ((e = prepare(k_edge_fwd_ws<KP, false, NSTG, WS_CH, WS_CE>, WS::BYTES))) return e;
-        e = launch_pdl(k_edge_fwd_ws<KP, false, NSTG, WS_CH, WS_CE>, dim3(G), dim3(WS_THREADS), WS::BYTES, s, a, NW);
+        static_assert(WS::ALLOC <= 227 * 1024, "shared memory plan exceeds 227 KB");
+        if ((e = prepare(k_edge_fwd_ws<KP, false, NSTG, WS_CH, WS_CE>, WS::ALLOC))) return e;
+        CUtensorMap xmap;
+        if ((e = a.t == 0 ? make_row_map(&xmap, a.emb, a.n_types)
+                          : make_row_map(&xmap, a.X + (int64_t)(a.t - 1) * a.N * FF, a.N)))
+            return e;
+        e = launch_pdl(k_edge_fwd_ws<KP, false, NSTG, WS_CH, WS_CE>, dim3(G), dim3(WS_THREADS), WS::ALLOC, s, a, NW,
+                       xmap);
     } else {
         if ((e = prepare(k_edge_fwd_tc<KP, SPLIT, NW, CH>, S::BYTES))) return e;
         e = launch_pdl(k_edge_fwd_tc<KP, SPLIT, NW, CH>, dim3(G), dim3(WGT * NW), S::BYTES, s, a);

@@ -192,6 +192,7 @@ struct EdgeTcArgs {
     float *Xbar;           // [N][F]
     float *forces;         // [N][3]
     int64_t N;
+    int n_types;           // rows of emb (the source rows of block 0)
     Geometry geo;
     Basis basis;
     const void *W1h, *W1l, *W2h, *W2l;

@@ -133,6 +133,21 @@ static __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, u
                  : "memory");
 }
 
+// Tensor-memory-accelerator gather (sm_100a): rows r0..r3 of the 2-D tensor described by the
+// tensor map at map (generic address of a __grid_constant__ parameter; boxes one row high,
+// starting at column x, which must be a multiple of 16 bytes' worth of elements) into four
+// consecutive box-sized rows of this CTA's shared memory at dst (128-byte aligned), completing
+// on mbar.  No multicast.
+static __device__ __forceinline__ void tma_gather4(uint32_t dst, const void *map, int x, int r0, int r1, int r2,
+                                                   int r3, uint32_t mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+        "l"(map), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(mbar)
+        : "memory");
+}
+
 // Bounded wait of the whole CTA for phase 0 of mbar (the weight copies); false on time-out.
 static __device__ __forceinline__ bool wait_copies(uint32_t mbar, int *d_err)
 {
