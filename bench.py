@@ -528,13 +528,13 @@ def run_ours(args):
 
     extras = {}
     if rank == 0 and world == 1 and not args.no_extras:
-        # the 4096-atom periodic box (cfg4) and the chains' evaluation alone, each mode; the
-        # whole-evaluation roofline of these and of the MD step timed above
+        # the chains' evaluation alone and the 4096- and 65,536-atom periodic boxes (cfg4,
+        # cfg5), each mode; the whole-evaluation roofline of these and of the MD step timed above
         extras["roofline_eval"] = {"cfg2_md_step": eval_roofline(m, N, E_mean, t_ms / args.steps / 1e3, pk, build=True)}
         extras["roofline_eval"]["cfg2_md_step"]["steps_x_replicas_per_s"] = value * R
         extras["roofline_eval"]["cfg2_md_step"]["roof_steps_x_replicas_per_s"] = \
             extras["roofline_eval"]["cfg2_md_step"]["roof_per_s"] * R
-        for cfg in (2, 4):
+        for cfg in (2, 4, 5):
             for name in ("fp16", "tc32"):
                 t_e, n_e, e_e, m_e = time_evals(cfg, PRECISIONS[name][0], 50, dev, stream, flush)
                 extras["roofline_eval"][f"cfg{cfg}_eval_{name}"] = eval_roofline(m_e, n_e, e_e, t_e, pk)

@@ -64,6 +64,7 @@ def report(what, gpu, ref, tol, bound_kind):
         if fr.function.startswith("test_"):
             rec["test"] = fr.function
             break
+    rec["case"] = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
     with open(path, "a") as f:
         f.write(json.dumps(rec) + "\n")
 
