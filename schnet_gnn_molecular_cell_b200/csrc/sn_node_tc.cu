@@ -40,7 +40,43 @@ struct NodeSmem {
     static constexpr uint32_t PR = HOLD + 16;       // float[64][TA] readout products (readout only)
     static constexpr uint32_t BYTES_UPDATE = PR;
     static constexpr uint32_t BYTES_READOUT = PR + 64 * TA * 4;
+    // update and backward with fp16 operands: the tile's two input row blocks, fp32 [TA][F]
+    // each, staged by bulk copies that complete on LB0 and LB1
+    static constexpr uint32_t LB0 = HOLD + 16;
+    static constexpr uint32_t LB1 = LB0 + 8;
+    static constexpr uint32_t IN0 = (LB1 + 8 + 127) / 128 * 128;
+    static constexpr uint32_t IN1 = IN0 + TA * FF * 4;
+    static constexpr uint32_t BYTES_STAGED = IN1 + TA * FF * 4;
 };
+
+// The input rows of a tile (na <= TA atoms from a0) into the staging blocks: thread 0 announces
+// the bytes on both barriers, then thread a copies row a of each input (512 bytes, 16-byte
+// aligned) -- row0(a) into IN0 (completing on LB0) and row1(a) into IN1 (on LB1).
+template <typename Row0, typename Row1>
+__device__ __forceinline__ void stage_rows(unsigned char *sm, int na, Row0 row0, Row1 row1)
+{
+    using S = NodeSmem<false>;
+    const uint32_t lb0 = smem_u32(sm + S::LB0), lb1 = smem_u32(sm + S::LB1);
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(lb0, (uint32_t)na * FF * 4);
+        mbar_expect_tx(lb1, (uint32_t)na * FF * 4);
+    }
+    __syncthreads();
+    if ((int)threadIdx.x < na) {
+        bulk_g2s(smem_u32(sm + S::IN0) + threadIdx.x * FF * 4, row0((int)threadIdx.x), FF * 4, lb0);
+        bulk_g2s(smem_u32(sm + S::IN1) + threadIdx.x * FF * 4, row1((int)threadIdx.x), FF * 4, lb1);
+    }
+}
+
+// Every thread waits, bounded, for one staging barrier's phase; false (and the time-out bit) if
+// the copies did not land.
+__device__ __forceinline__ bool staged(unsigned char *sm, uint32_t off, uint32_t parity, int *d_err)
+{
+    int ok = bounded_phase_wait(smem_u32(sm + off), parity, 1ll << 33);
+    ok = __syncthreads_and(ok);
+    if (!ok && threadIdx.x == 0) atomicOr(d_err, ERRBIT_TIMEOUT);
+    return ok != 0;
+}
 
 // D[o][a] = sum_i W[o][i] T[a][i]  (TRANS = false)  or  D[i][a] = sum_o W[o][i] T[a][o]  (TRANS)
 template <bool SPLIT, bool TRANS>
@@ -122,7 +158,7 @@ __device__ __forceinline__ const float *x_row(const NodeTcArgs &A, int t, int64_
     return A.X + ((int64_t)(t - 1) * A.N + a) * FF;
 }
 
-template <bool SPLIT>
+template <bool SPLIT, bool STAGED = false>
 __device__ __forceinline__ uint32_t node_setup(const NodeTcArgs &A, unsigned char *sm, const void *w0h,
                                                const void *w0l, const void *w1h, const void *w1l, int &skip)
 {
@@ -131,6 +167,10 @@ __device__ __forceinline__ uint32_t node_setup(const NodeTcArgs &A, unsigned cha
     if (threadIdx.x == 0) {
         mbar_init(smem_u32(sm + S::MBAR), 1);
         mbar_init(wmbar, 1);
+        if (STAGED) {
+            mbar_init(smem_u32(sm + NodeSmem<false>::LB0), 1);
+            mbar_init(smem_u32(sm + NodeSmem<false>::LB1), 1);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         mbar_expect_tx(wmbar, S::NS * S::WB * (w1h ? 2 : 1));   // constant weights: before the wait
         bulk_g2s(smem_u32(sm + S::W0), w0h, S::WB, wmbar);
@@ -167,7 +207,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
     using S = NodeSmem<SPLIT>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
-    const uint32_t tmem = node_setup<SPLIT>(A, sm, A.U1h, A.U1l, A.U2h, A.U2l, skip);
+    const uint32_t tmem = node_setup<SPLIT, !SPLIT>(A, sm, A.U1h, A.U1l, A.U2h, A.U2l, skip);
     const int f = threadIdx.x % WGT, g = threadIdx.x / WGT, c = g;
     const uint32_t lane = (uint32_t)((f >> 5) * 32) << 16;
     const uint32_t mbar = smem_u32(sm + S::MBAR);
@@ -179,16 +219,29 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
         const float c1f = A.c1[f], c2f = A.c2[f], su1f = A.su1[f], su2f = A.su2[f];
         unsigned char *T = sm + S::T;
         bool ok = true;
+        bool pending = false;   // the second input of a tile copied but not yet waited for
+        uint32_t sp = 0;        // parity of this tile's staging barriers
         for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            sp = (uint32_t)(((tile - blockIdx.x) / gridDim.x) & 1);
             const int64_t a0 = tile * TA, ab = a0 + 32 * c;   // this thread's atoms: ab + q, q < nv
             const int nv = chunk_atoms(a0, c, A.N);
             const float *Hp = A.H + ab * FF + f;
             float *Pp = A.P + ((int64_t)A.t * A.N + ab) * FF + f;
             float *Xp = A.X + ((int64_t)A.t * A.N + ab) * FF + f;
-            tile_from<SPLIT>(T, f, g, nv, [&](int q) { return Hp[q * FF]; });
-            float xr[32];   // the residual's x^t, loaded while the GEMMs run
+            float xr[32];   // the residual's x^t
+            if constexpr (SPLIT) {
+                tile_from<SPLIT>(T, f, g, nv, [&](int q) { return Hp[q * FF]; });
 #pragma unroll
-            for (int q = 0; q < 32; ++q) xr[q] = q < nv ? ldnc_keep(x_row(A, A.t, ab + q) + f) : 0.0f;
+                for (int q = 0; q < 32; ++q) xr[q] = q < nv ? ldnc_keep(x_row(A, A.t, ab + q) + f) : 0.0f;
+            } else {   // h and x^t rows of the tile by bulk copies (x^t waited for at its use)
+                const int na = (int)(A.N - a0 < TA ? A.N - a0 : TA);
+                stage_rows(sm, na, [&](int a) { return A.H + (a0 + a) * FF; },
+                           [&](int a) { return x_row(A, A.t, a0 + a); });
+                pending = true;
+                if (!(ok = staged(sm, S::LB0, sp, A.d_err))) break;
+                const float *sH = reinterpret_cast<const float *>(sm + S::IN0) + 32 * c * FF + f;
+                tile_from<SPLIT>(T, f, g, nv, [&](int q) { return sH[q * FF]; });
+            }
             if (!(ok = gemm_step<SPLIT, false>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
             {
                 float v[32];
@@ -202,6 +255,13 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
                 store_tile_col<SPLIT, 32>(T, T + S::TB, f, 32 * c, v);
             }
             if (!(ok = gemm_step<SPLIT, false>(sm + S::W1, T, tmem + 128, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
+            if constexpr (!SPLIT) {
+                if (!(ok = staged(sm, S::LB1, sp, A.d_err))) break;
+                pending = false;
+                const float *sX = reinterpret_cast<const float *>(sm + S::IN1) + 32 * c * FF + f;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) xr[q] = q < nv ? sX[q * FF] : 0.0f;
+            }
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 128 + 32 * c, v);
@@ -212,7 +272,10 @@ __global__ void __launch_bounds__(NT, 1) k_node_update_tc(NodeTcArgs A)
             tc_fence_before();
             __syncthreads();
         }
-        if (!ok) drain_cta(mbar, phase, A.d_err);
+        if (!ok) {
+            drain_cta(mbar, phase, A.d_err);
+            if (!SPLIT && pending) staged(sm, NodeSmem<false>::LB1, sp, A.d_err);   // no copy left in flight
+        }
     }
     node_teardown(tmem, ready, wmbar, A.d_err);
 }
@@ -291,7 +354,7 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
     using S = NodeSmem<SPLIT>;
     extern __shared__ __align__(128) unsigned char sm[];
     __shared__ int skip;
-    const uint32_t tmem = node_setup<SPLIT>(A, sm, A.U2h, A.U2l, A.U1h, A.U1l, skip);
+    const uint32_t tmem = node_setup<SPLIT, !SPLIT>(A, sm, A.U2h, A.U2l, A.U1h, A.U1l, skip);
     const int f = threadIdx.x % WGT, g = threadIdx.x / WGT, c = g;
     const uint32_t lane = (uint32_t)((f >> 5) * 32) << 16;
     const uint32_t mbar = smem_u32(sm + S::MBAR);
@@ -304,16 +367,36 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
         // the operands of U2^T and U1^T carry the channel scales of U2 and U1
         const float su1f = A.su1[f], su2f = A.su2[f];
         bool ok = true;
+        bool pending = false;   // the second input of a tile copied but not yet waited for
+        uint32_t sp = 0;        // parity of this tile's staging barriers
         for (int64_t tile = blockIdx.x; tile < n_tiles && ok; tile += gridDim.x) {
+            sp = (uint32_t)(((tile - blockIdx.x) / gridDim.x) & 1);
             const int64_t a0 = tile * TA, ab = a0 + 32 * c;
             const int nv = chunk_atoms(a0, c, A.N);
             const float *Bp = A.Xbar + ab * FF + f;
             const float *Pp = A.P + ((int64_t)A.t * A.N + ab) * FF + f;
-            tile_from<SPLIT>(T, f, g, nv, [&](int q) { return Bp[q * FF] * su2f; });
-            float pr[32];   // p of this thread's atoms, loaded while the first GEMM runs
+            float pr[32];   // p of this thread's atoms
+            if constexpr (SPLIT) {
+                tile_from<SPLIT>(T, f, g, nv, [&](int q) { return Bp[q * FF] * su2f; });
 #pragma unroll
-            for (int q = 0; q < 32; ++q) pr[q] = q < nv ? ldnc_keep(Pp + q * FF) : 0.0f;
+                for (int q = 0; q < 32; ++q) pr[q] = q < nv ? ldnc_keep(Pp + q * FF) : 0.0f;
+            } else {   // xbar and p rows of the tile by bulk copies (p waited for at its use)
+                const int na = (int)(A.N - a0 < TA ? A.N - a0 : TA);
+                stage_rows(sm, na, [&](int a) { return A.Xbar + (a0 + a) * FF; },
+                           [&](int a) { return A.P + ((int64_t)A.t * A.N + a0 + a) * FF; });
+                pending = true;
+                if (!(ok = staged(sm, S::LB0, sp, A.d_err))) break;
+                const float *sB = reinterpret_cast<const float *>(sm + S::IN0) + 32 * c * FF + f;
+                tile_from<SPLIT>(T, f, g, nv, [&](int q) { return sB[q * FF] * su2f; });
+            }
             if (!(ok = gemm_step<SPLIT, true>(sm + S::W0, T, tmem, mbar, phase, A.d_err, ready, wmbar, A.wait_limit))) break;
+            if constexpr (!SPLIT) {
+                if (!(ok = staged(sm, S::LB1, sp, A.d_err))) break;
+                pending = false;
+                const float *sP = reinterpret_cast<const float *>(sm + S::IN1) + 32 * c * FF + f;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) pr[q] = q < nv ? sP[q * FF] : 0.0f;
+            }
             {
                 float v[32];
                 tmem_ld32(tmem + lane + 32 * c, v);
@@ -333,7 +416,10 @@ __global__ void __launch_bounds__(NT, 1) k_node_bwd_tc(NodeTcArgs A)
             tc_fence_before();
             __syncthreads();
         }
-        if (!ok) drain_cta(mbar, phase, A.d_err);
+        if (!ok) {
+            drain_cta(mbar, phase, A.d_err);
+            if (!SPLIT && pending) staged(sm, NodeSmem<false>::LB1, sp, A.d_err);   // no copy left in flight
+        }
     }
     node_teardown(tmem, ready, wmbar, A.d_err);
 }
@@ -361,9 +447,10 @@ cudaError_t launch_node_tc(const NodeTcArgs &a, bool split, int which, int n_sm,
         return launch_k(k_node_bwd_tc<true>, S::BYTES_UPDATE, grid, a, s);
     }
     using S = NodeSmem<false>;
-    if (which == 0) return launch_k(k_node_update_tc<false>, S::BYTES_UPDATE, grid, a, s);
+    static_assert(S::BYTES_STAGED <= 227 * 1024, "shared memory plan exceeds 227 KB");
+    if (which == 0) return launch_k(k_node_update_tc<false>, S::BYTES_STAGED, grid, a, s);
     if (which == 1) return launch_k(k_node_readout_tc<false>, S::BYTES_READOUT, grid, a, s);
-    return launch_k(k_node_bwd_tc<false>, S::BYTES_UPDATE, grid, a, s);
+    return launch_k(k_node_bwd_tc<false>, S::BYTES_STAGED, grid, a, s);
 }
 
 }  // namespace sn

@@ -254,3 +254,46 @@ def test_md_tensor_modes_match_oracle(oracle, dev, cfg, precision, integrator):
     check(energy.cpu().numpy(), E_o, f"energy at final positions ({integrator})")
     check(forces.cpu().numpy(), F_o, f"forces at final positions ({integrator})")
     assert ctx.md_edges() == len(cl)
+
+
+@pytest.mark.parametrize("precision,factor", [(2, 1.25), (1, 10.0)], ids=["tc32", "fp16"])
+def test_nve_drift_matches_oracle(oracle, dev, precision, factor):
+    """cfg3 (the chains as NVE velocity Verlet at 2 fs, 12 amu): the total-energy drift of
+    replicas 0-3 over 100 GPU steps, max_t |E(t) - E(0)| / (n k_B T), against the oracle's
+    double-precision drift from the same start.  At 2 fs the drift is the integrator's, so
+    the fp32-accurate mode must reproduce the oracle's within 25 %; fp16 operands add energy
+    noise of their own (about 4x the oracle's drift at this step), bounded at 10x."""
+    from schnet_gnn_molecular_cell_b200 import Context
+    steps, n_rep, mass, dt = 100, 4, 12.0, 2.0
+    w = synth.make_workload(2)
+    s, m = w.system, w.model
+    n = s.n_per_replica
+    v0 = synth.maxwell_boltzmann(n, s.n_replicas, mass, 300.0, seed=4002)
+    kin0 = lambda v, r: 0.5 * mass / synth.KAPPA * (v.astype(np.float64).reshape(r, n, 3) ** 2).sum(axis=(1, 2))  # noqa: E731
+    key = ("drift", steps, n_rep)
+    if key not in _ORACLE_TRAJ:
+        so = synth.SystemCfg(n, n_rep, s.box)
+        po, vo, ty = w.pos[: n * n_rep], v0[: n * n_rep], w.types[: n * n_rep]
+        _, _, _, epot, ekin, _ = oracle.md_vv(m, w.weights, so, po, vo, ty, mass, dt, steps)
+        rp, cl = oracle.neighbors(so, m.r_cut, po)
+        e0, _, _ = oracle.energy_forces(m, w.weights, so, po, ty, rp, cl)
+        _ORACLE_TRAJ[key] = np.vstack([e0 + kin0(vo, n_rep), epot + ekin])
+    et_o = _ORACLE_TRAJ[key]
+    ctx = Context(m, w.weights, precision=precision)
+    pos = torch.from_numpy(w.pos.copy()).to(dev)
+    vel = torch.from_numpy(v0.copy()).to(dev)
+    types = torch.from_numpy(w.types).to(dev)
+    rp, cl = ctx.neighbors(s, pos)
+    e0, forces = ctx.energy_forces(s, pos, types, rp, cl)
+    forces = forces.clone()
+    hist = torch.empty((steps, 2, s.n_replicas), device=dev)
+    for k in range(steps):
+        ctx.md_step(s, pos, vel, forces, types, mass, dt, 1, hist[k, 0], hist[k, 1])
+    ctx.sync()
+    h = hist.double().cpu().numpy()
+    et_g = np.vstack([e0.double().cpu().numpy() + kin0(v0, s.n_replicas), h[:, 0] + h[:, 1]])[:, :n_rep]
+    kT = synth.KB * 300.0
+    d_o = np.abs(et_o - et_o[:1]).max(axis=0) / (n * kT)
+    d_g = np.abs(et_g - et_g[:1]).max(axis=0) / (n * kT)
+    assert np.all(d_g < 1e-3), d_g
+    assert np.all(d_g <= factor * d_o + 1e-7), (d_g.tolist(), d_o.tolist())
