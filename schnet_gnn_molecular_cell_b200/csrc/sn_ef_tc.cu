@@ -927,10 +927,14 @@ __global__ void __launch_bounds__(WS_THREADS, 1)
     if (!skip && r0 < r1) {
         if (warp >= WS_P_WARP0 && warp < WS_M_WARP) {
             // P: the prologue of tile k (edge n = t % 64, a quarter of its Gaussians per
-            // thread), with tile k + 1's indices and positions read ahead
+            // thread), with tile k + 1's indices and positions read ahead by part 0 (t < 64),
+            // the only part that uses them (metadata, row starts, gathers); the other parts
+            // take d and C(d) from the stage
             const int t = threadIdx.x - 32 * WS_P_WARP0, nf = t & (TE - 1);
-            EdgeIdx nidx = load_idx(A, e0 + nf, e1);
-            EdgePos npos = load_pos(A, nidx);
+            const int e_lim = t < TE ? e1 : 0;   // (load_idx gives zeros at or past e_lim)
+            EdgeIdx nidx = load_idx(A, e0 + nf, e_lim);
+            EdgePos npos{};
+            if (t < TE) npos = load_pos(A, nidx);
             for (int k = 0; k < nt; ++k) {
                 const int s = k % NSTG, ts = e0 + k * TE, ne = min(TE, e1 - ts);
                 int okw = 1;
@@ -938,7 +942,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1)
                 if (!named_sync_and(5, WS_P, okw)) break;   // all P warps go on or stop together
                 const EdgeIdx cidx = nidx;
                 const EdgePos cpos = npos;
-                if (k + 1 < nt) nidx = load_idx(A, ts + TE + nf, e1);
+                if (k + 1 < nt) nidx = load_idx(A, ts + TE + nf, e_lim);
                 if (t < 64) {
                     // source rows first, so that they land during the prologue: lane 4 g of P
                     // warp w (0 or 1) gathers the rows of edges 32 w + 4 g + [0, 4), which lanes
@@ -959,7 +963,7 @@ __global__ void __launch_bounds__(WS_THREADS, 1)
                 tile_prologue<S, KP, SPLIT, false, 4, true>(A, sm, stage(s), t, ts, ne, cidx, cpos);
                 fence_async_smem();
                 mbar_arrive(bar(WB_FULL_B, s));
-                if (k + 1 < nt) npos = load_pos(A, nidx);
+                if (k + 1 < nt && t < TE) npos = load_pos(A, nidx);
             }
         } else if (warp == WS_M_WARP) {
             // M: lane 0 polls the two queues and issues whichever MMA is ready: MMA1 of the next

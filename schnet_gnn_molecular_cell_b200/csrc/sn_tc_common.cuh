@@ -234,28 +234,13 @@ static __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8])
     for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// This lane's 4 consecutive 32-bit TMEM columns starting at taddr.
-static __device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4])
-{
-    uint32_t r[4];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-        : "r"(taddr)
-        : "memory");
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
-}
-
 template <int CH>
 static __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[CH])
 {
-    static_assert(CH == 4 || CH == 8 || CH == 16 || CH == 32, "4, 8, 16 or 32 columns");
+    static_assert(CH == 8 || CH == 16 || CH == 32, "8, 16 or 32 columns");
     if constexpr (CH == 32) tmem_ld32(taddr, v);
     else if constexpr (CH == 16) tmem_ld16(taddr, v);
-    else if constexpr (CH == 8) tmem_ld8(taddr, v);
-    else tmem_ld4(taddr, v);
+    else tmem_ld8(taddr, v);
 }
 
 // 16 lanes x 64 bits, 16 repetitions: thread t of the warp receives lane 8 (t % 2) + t / 4 of
